@@ -1,0 +1,165 @@
+/* wal.h -- C ABI of libwal.so: the direct-packed body-matrix product on B200.
+ *
+ *   y = (alpha * T + beta * R) x + sum_r s_r U_r (V_r^T x)
+ *
+ * The product, its parts and their names follow the WAL-Ternary-8B model card
+ * (section "Representation"; the Kazakh README, section "Model format", prints
+ * the same formula):
+ *   T      ternary base, T in {-1, 0, +1}, stored as packed 2-bit codes
+ *          (32 bytes per 128 weights with three of four codes used, like PQ2_0
+ *          on the WAL2-Ternary-27B card, section on bit widths);
+ *   R      exactly k signed residual sites per group of 128 weights, k in
+ *          {0, 2, 4, 8} (WAL-Ternary-27B-RC1 card, "Representation": k0/k2/k4/k8);
+ *   alpha, beta  FP16 scales per (output row, 128-group) (WAL-Ternary-8B card,
+ *          "Install": the cache keeps FP16 scales; the 128-weight scale group
+ *          is the WAL2-Ternary-27B card's, "Архитектура");
+ *   U, V   the WALB2 binary low-rank pair, entries +-1, with one FP16 scale per
+ *          rank (WAL-Ternary-8B card, "Representation": packed binary low-rank
+ *          WALB2 correction).
+ *
+ * Layout v1 (the byte format every entry point reads), N outputs, K inputs,
+ * G = K / 128 groups, k sites per group, rank r:
+ *   codes    uint32[N][K/16]   trit j of row n in word j/16, bits 2*(j%16)..+1;
+ *                              code c = t + 1 (0 -> -1, 1 -> 0, 2 -> +1), 3 reserved
+ *   sites    uint8 [N][G][k]   byte = position in group (bits 0..6) | 0x80 if the
+ *                              site's sign is -1; positions distinct, ascending
+ *   scales   uint16[N][G][2]   fp16 bits {alpha, beta} when k > 0;
+ *            uint16[N][G]      fp16 bits alpha when k == 0
+ *   u_bits   uint32[N][ceil(r/32)]  bit (rho % 32) of word rho/32 set <=> U[n][rho] = -1
+ *   v_bits   uint32[r][K/32]   bit (j % 32) of word j/32 set <=> V[j][rho] = -1
+ *   lr_scale uint16[r]         fp16 bits of s_rho
+ * Activations are bf16 bit patterns, row-major X[M][ldx]; outputs are fp32,
+ * row-major Y[M][ldy], overwritten (never accumulated into).
+ *
+ * Conventions for every entry point:
+ *   - Ownership: the caller owns every buffer.  The library never allocates
+ *     device memory; scratch comes from the caller as (ws, ws_bytes), sized by
+ *     the matching *_workspace_bytes call.  Plans own only a CUDA graph.
+ *   - Matrix buffers and activations must be 16-byte aligned, outputs 4-byte
+ *     aligned; otherwise WAL_ERR_ARG.
+ *   - Stream semantics: device work is enqueued on `stream` and returns at
+ *     once; argument and shape errors are returned synchronously before any
+ *     launch.  Launch failures return WAL_ERR_CUDA.  A bounded wait inside a
+ *     kernel that gives up records WAL_ERR_TIMEOUT in the workspace header,
+ *     which wal_device_status() reads.
+ *   - No exceptions and no aborts cross the ABI.  wal_last_error() returns a
+ *     thread-local text for the last non-OK status of the calling thread.
+ *   - There is no CPU fallback: every device entry point runs CUDA kernels
+ *     built for sm_100a and fails with WAL_ERR_CUDA when no such device exists.
+ */
+#ifndef WAL_H
+#define WAL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st* wal_stream_t;
+
+enum {
+  WAL_OK = 0,
+  WAL_ERR_ARG = -1,         /* null / misaligned pointer, bad count */
+  WAL_ERR_SHAPE = -2,       /* K % 128 != 0, k not in {0,2,4,8}, r > 32, N <= 0, M out of range */
+  WAL_ERR_FORMAT = -3,      /* buffer content violates layout v1 */
+  WAL_ERR_WORKSPACE = -4,   /* ws_bytes smaller than required */
+  WAL_ERR_CUDA = -5,        /* a CUDA runtime call failed */
+  WAL_ERR_UNSUPPORTED = -6, /* valid but not handled by this build */
+  WAL_ERR_TIMEOUT = -7      /* a bounded device wait gave up */
+};
+
+#define WAL_MAX_RANK 32
+#define WAL_MAX_SMALL_M 16
+
+/* One packed matrix.  All pointers are device pointers into caller-owned
+ * buffers laid out as described above; `sites` may be NULL when k == 0 and
+ * `u_bits`, `v_bits`, `lr_scale` may be NULL when r == 0. */
+typedef struct wal_matrix {
+  int32_t N, K, k, r;
+  const uint32_t* codes;
+  const uint8_t* sites;
+  const uint16_t* scales;
+  const uint32_t* u_bits;
+  const uint32_t* v_bits;
+  const uint16_t* lr_scale;
+} wal_matrix;
+
+/* Byte sizes of the six layout-v1 buffers, in the order codes, sites, scales,
+ * u_bits, v_bits, lr_scale.  Host only.  WAL_ERR_SHAPE on a bad shape. */
+int wal_packed_sizes(int N, int K, int k, int r, size_t out_bytes[6]);
+
+/* Pack dense components (host arrays) into the six layout-v1 buffers (host
+ * memory, sizes from wal_packed_sizes).  Inputs:
+ *   T [N][K] int8 in {-1,0,1}; site_pos [N][G][k] uint8 < 128, strictly
+ *   ascending per group; site_sign [N][G][k] int8 +-1; alpha, beta [N][G]
+ *   fp16 bits (beta ignored and may be NULL when k == 0); U [N][r] and
+ *   V [K][r] int8 +-1; lr_scale [r] fp16 bits.
+ * Host only, multi-threaded.  WAL_ERR_FORMAT on any out-of-range value;
+ * nothing is guaranteed about out[] then. */
+int wal_pack_matrix(const int8_t* T, const uint8_t* site_pos, const int8_t* site_sign,
+                    const uint16_t* alpha, const uint16_t* beta, const int8_t* U,
+                    const int8_t* V, const uint16_t* lr_scale, int N, int K, int k, int r,
+                    void* const out[6]);
+
+/* Scan a packed matrix on the device for layout-v1 violations (reserved code
+ * 3, site positions not strictly ascending).  Synchronises `stream`.
+ * Returns WAL_OK or WAL_ERR_FORMAT (wal_last_error names the first kind found).
+ * ws must hold at least 256 bytes. */
+int wal_validate(const wal_matrix* m, void* ws, size_t ws_bytes, wal_stream_t stream);
+
+/* Test entry point: decode a packed matrix on the device into dense device
+ * arrays with the same decode routines the product kernels use.
+ *   T [N][K] int8; site_pos, site_sign [N][G][k]; alpha, beta [N][G] fp16 bits
+ *   (beta zero-filled when k == 0); U [N][r] int8; V [K][r] int8.
+ * Any output pointer may be NULL to skip it.  Asynchronous. */
+int wal_unpack_matrix(const wal_matrix* m, int8_t* T, uint8_t* site_pos, int8_t* site_sign,
+                      uint16_t* alpha, uint16_t* beta, int8_t* U, int8_t* V,
+                      wal_stream_t stream);
+
+/* Scratch bytes wal_gemv (M = 1) / wal_gemm_small_m (M <= 16) need. */
+size_t wal_workspace_bytes(const wal_matrix* m, int M);
+
+/* y[N] = W x for one bf16 activation x[K] (batch 1): the decode-GEMV.
+ * Streams the packed planes once, FP32 output. */
+int wal_gemv(const wal_matrix* m, const uint16_t* x, float* y, void* ws, size_t ws_bytes,
+             wal_stream_t stream);
+
+/* Y[M][ldy] = X[M][ldx] W^T for 1 <= M.  M <= 16 runs the CUDA-core
+ * decode-GEMV family with M accumulators per row; M >= 64 runs the tensor-core
+ * path (TMA + tcgen05).  ldx >= K and a multiple of 8; ldy >= N. */
+int wal_gemm_small_m(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, int ldy,
+                     void* ws, size_t ws_bytes, wal_stream_t stream);
+
+/* Read and clear the device status word in a workspace header (synchronises
+ * `stream`).  Every product call clears the word when it starts, so it reports
+ * on the last call that used this workspace.  WAL_OK or WAL_ERR_TIMEOUT. */
+int wal_device_status(void* ws, wal_stream_t stream);
+
+/* Whole body pass: n_mats products, matrix i reading xs[i] (bf16 [M][K_i]) and
+ * writing ys[i] (fp32 [M][N_i]).  stage_of[i] is the dependency stage of
+ * matrix i: all matrices of stage s may run concurrently, and stage s + 1
+ * starts only after every product of stage s has finished (a matrix of a
+ * later stage may read an output of an earlier one).  Stages must be
+ * non-decreasing along the array.  mats, stage_of, xs and ys are host arrays
+ * (of device pointers).
+ * The first call builds *plan (a CUDA graph of the pass on `stream`); later
+ * calls with identical arguments replay it.  A call whose arguments differ
+ * from the plan's rebuilds it. */
+typedef struct wal_body_plan wal_body_plan;
+size_t wal_body_workspace_bytes(const wal_matrix* mats, int n_mats, int M);
+int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n_mats,
+                  const int32_t* stage_of, const uint16_t* const* xs, float* const* ys, int M,
+                  void* ws, size_t ws_bytes, wal_stream_t stream);
+void wal_body_plan_destroy(wal_body_plan* plan);
+
+const char* wal_status_string(int status);
+const char* wal_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WAL_H */

@@ -9,6 +9,7 @@ from .wal_oracle import (  # noqa: F401
     pack,
     unpack,
     packed_sizes,
+    payload_sizes,
     bits_per_weight,
     dense_weight,
     matvec,

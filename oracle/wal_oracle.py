@@ -29,6 +29,7 @@ reason in the design notes):
 * WALB2: y += sum_r s_r * U[:, r] * (V[:, r]^T x) with one FP16 scale s_r per
   rank; U, V in {+1, -1}; a set bit means -1.  U is stored as
   u32[N][ceil(r/32)], V as u32[r][K/32].
+* every buffer is zero-padded to a multiple of 16 bytes.
 
 Every float is widened exactly (fp16 / bf16 -> float64) and W is formed
 densely in float64; y = W x is one float64 matrix product.  There is no
@@ -77,8 +78,9 @@ def _check_shape(N, K, k, r):
         raise FormatError(f"r={r} outside [0, {MAX_RANK}]")
 
 
-def packed_sizes(N: int, K: int, k: int, r: int):
-    """Byte size of the six layout-v1 buffers: codes, sites, scales, U bits, V bits, s."""
+def payload_sizes(N: int, K: int, k: int, r: int):
+    """Bytes of information in the six layout-v1 buffers: codes, sites, scales,
+    U bits, V bits, s (before padding)."""
     _check_shape(N, K, k, r)
     G = K // GROUP
     codes = N * K // 4
@@ -90,8 +92,13 @@ def packed_sizes(N: int, K: int, k: int, r: int):
     return [codes, sites, scales, ubits, vbits, lr]
 
 
+def packed_sizes(N: int, K: int, k: int, r: int):
+    """Allocated size of each buffer: the payload zero-padded to a multiple of 16 bytes."""
+    return [(s + 15) // 16 * 16 for s in payload_sizes(N, K, k, r)]
+
+
 def bits_per_weight(N: int, K: int, k: int, r: int) -> float:
-    return 8.0 * sum(packed_sizes(N, K, k, r)) / (N * K)
+    return 8.0 * sum(payload_sizes(N, K, k, r)) / (N * K)
 
 
 # ---------------------------------------------------------------------------
@@ -155,8 +162,13 @@ def pack(c) -> list:
     vbits = np.bitwise_or.reduce(vneg << np.arange(32, dtype=np.uint32), axis=2).astype(np.uint32) \
         if r else np.zeros((0, K // 32), np.uint32)
     lr = np.asarray(c.lr_scale, dtype=np.uint16).reshape(r).copy()
-    return [codes.reshape(-1), sites.reshape(-1), scales.reshape(-1), ubits.reshape(-1),
-            vbits.reshape(-1), lr]
+    out = []
+    for b, size in zip([codes, sites, scales, ubits, vbits, lr], packed_sizes(N, K, k, r)):
+        raw = np.zeros(size, dtype=np.uint8)
+        bb = np.ascontiguousarray(b).reshape(-1).view(np.uint8)
+        raw[: bb.size] = bb
+        out.append(raw)
+    return out
 
 
 def _as_u8(buf) -> np.ndarray:
@@ -171,10 +183,14 @@ def unpack(bufs, N: int, K: int, k: int, r: int) -> Unpacked:
     _check_shape(N, K, k, r)
     G = K // GROUP
     sizes = packed_sizes(N, K, k, r)
+    used = payload_sizes(N, K, k, r)
     raw = [_as_u8(b) for b in bufs]
-    for i, (b, s) in enumerate(zip(raw, sizes)):
+    for i, (b, s, u) in enumerate(zip(raw, sizes, used)):
         if b.size != s:
             raise FormatError(f"buffer {i} has {b.size} bytes, expected {s}")
+        if np.any(b[u:]):
+            raise FormatError(f"buffer {i} has nonzero padding")
+    raw = [b[:u] for b, u in zip(raw, used)]
     words = raw[0].view('<u4').reshape(N, K // 16, 1)
     code = (words >> (2 * np.arange(16, dtype=np.uint32))) & 3
     if np.any(code == 3):
@@ -202,7 +218,7 @@ def unpack(bufs, N: int, K: int, k: int, r: int) -> Unpacked:
     vb = raw[4].view('<u4').reshape(r, K // 32) if r else np.zeros((0, K // 32), np.uint32)
     vneg = (vb[:, :, None] >> np.arange(32, dtype=np.uint32)) & 1
     V = np.where(vneg.reshape(r, K).T, -1, 1).astype(np.int8) if r else np.zeros((K, 0), np.int8)
-    lr = raw[5].view('<u2').copy()
+    lr = raw[5].view('<u2').copy() if r else np.zeros(0, np.uint16)
     return Unpacked(N, K, k, r, T, pos, sgn, alpha, beta, U, V, lr)
 
 

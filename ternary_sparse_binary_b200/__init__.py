@@ -1,0 +1,16 @@
+"""B200-native direct-packed body-matrix product (libwal.so) -- Python binding.
+
+The binding only marshals arguments into the C ABI declared in include/wal.h;
+every step of the product runs in the library's CUDA kernels.  PyTorch is
+used for device memory and streams.  There is no CPU fallback: if libwal.so
+cannot be loaded, importing this package raises.
+"""
+from ._abi import (  # noqa: F401
+    WAL_OK, WAL_ERR_ARG, WAL_ERR_SHAPE, WAL_ERR_FORMAT, WAL_ERR_WORKSPACE, WAL_ERR_CUDA,
+    WAL_ERR_UNSUPPORTED, WAL_ERR_TIMEOUT, WAL_MAX_RANK, WAL_MAX_SMALL_M,
+    WalError, wal_matrix, lib, lib_path, EXPORTED_SYMBOLS,
+    wal_packed_sizes, wal_pack_matrix, wal_validate, wal_unpack_matrix, wal_workspace_bytes,
+    wal_gemv, wal_gemm_small_m, wal_device_status, wal_body_workspace_bytes, wal_body_pass,
+    wal_body_plan_destroy, wal_status_string, wal_last_error,
+)
+from .packed import PackedMatrix, pack_host, to_device, BodyPass  # noqa: F401

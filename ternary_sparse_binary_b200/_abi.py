@@ -1,0 +1,146 @@
+"""ctypes declarations of the libwal.so C ABI (include/wal.h), same names.
+
+Every function takes plain integers for pointers (host pointers from numpy,
+device pointers from torch ``data_ptr()``), raises ``WalError`` on a non-OK
+status and otherwise returns what the C function returns.
+"""
+import ctypes
+import os
+
+from .build import LIB, build
+
+WAL_OK = 0
+WAL_ERR_ARG = -1
+WAL_ERR_SHAPE = -2
+WAL_ERR_FORMAT = -3
+WAL_ERR_WORKSPACE = -4
+WAL_ERR_CUDA = -5
+WAL_ERR_UNSUPPORTED = -6
+WAL_ERR_TIMEOUT = -7
+WAL_MAX_RANK = 32
+WAL_MAX_SMALL_M = 16
+
+EXPORTED_SYMBOLS = [
+    "wal_packed_sizes", "wal_pack_matrix", "wal_validate", "wal_unpack_matrix",
+    "wal_workspace_bytes", "wal_gemv", "wal_gemm_small_m", "wal_device_status",
+    "wal_body_workspace_bytes", "wal_body_pass", "wal_body_plan_destroy",
+    "wal_status_string", "wal_last_error",
+]
+
+
+class WalError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {wal_status_string(status)} ({wal_last_error()})")
+
+
+class wal_matrix(ctypes.Structure):
+    _fields_ = [
+        ("N", ctypes.c_int32), ("K", ctypes.c_int32), ("k", ctypes.c_int32), ("r", ctypes.c_int32),
+        ("codes", ctypes.c_void_p), ("sites", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+        ("u_bits", ctypes.c_void_p), ("v_bits", ctypes.c_void_p), ("lr_scale", ctypes.c_void_p),
+    ]
+
+
+def _load():
+    path = LIB if os.path.exists(LIB) else build()
+    return ctypes.CDLL(path)
+
+
+lib = _load()
+lib_path = LIB
+
+_vp, _sz, _i = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+_MP = ctypes.POINTER(wal_matrix)
+
+lib.wal_packed_sizes.argtypes = [_i, _i, _i, _i, ctypes.POINTER(_sz)]
+lib.wal_pack_matrix.argtypes = [_vp] * 8 + [_i] * 4 + [ctypes.POINTER(_vp)]
+lib.wal_validate.argtypes = [_MP, _vp, _sz, _vp]
+lib.wal_unpack_matrix.argtypes = [_MP] + [_vp] * 7 + [_vp]
+lib.wal_workspace_bytes.argtypes = [_MP, _i]
+lib.wal_workspace_bytes.restype = _sz
+lib.wal_gemv.argtypes = [_MP, _vp, _vp, _vp, _sz, _vp]
+lib.wal_gemm_small_m.argtypes = [_MP, _vp, _i, _i, _vp, _i, _vp, _sz, _vp]
+lib.wal_device_status.argtypes = [_vp, _vp]
+lib.wal_body_workspace_bytes.argtypes = [_MP, _i, _i]
+lib.wal_body_workspace_bytes.restype = _sz
+lib.wal_body_pass.argtypes = [ctypes.POINTER(_vp), _MP, _i, ctypes.POINTER(ctypes.c_int32),
+                              ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp, _sz, _vp]
+lib.wal_body_plan_destroy.argtypes = [_vp]
+lib.wal_body_plan_destroy.restype = None
+lib.wal_status_string.argtypes = [_i]
+lib.wal_status_string.restype = ctypes.c_char_p
+lib.wal_last_error.argtypes = []
+lib.wal_last_error.restype = ctypes.c_char_p
+
+
+def wal_status_string(status):
+    return lib.wal_status_string(int(status)).decode()
+
+
+def wal_last_error():
+    return lib.wal_last_error().decode()
+
+
+def _check(status, where):
+    if status != WAL_OK:
+        raise WalError(status, where)
+    return status
+
+
+def wal_packed_sizes(N, K, k, r):
+    out = (_sz * 6)()
+    _check(lib.wal_packed_sizes(N, K, k, r, out), "wal_packed_sizes")
+    return [int(v) for v in out]
+
+
+def wal_pack_matrix(T, site_pos, site_sign, alpha, beta, U, V, lr_scale, N, K, k, r, out):
+    arr = (_vp * 6)(*[int(p) if p else None for p in out])
+    return _check(lib.wal_pack_matrix(T, site_pos, site_sign, alpha, beta, U, V, lr_scale,
+                                      N, K, k, r, arr), "wal_pack_matrix")
+
+
+def wal_validate(m, ws, ws_bytes, stream):
+    return _check(lib.wal_validate(ctypes.byref(m), ws, ws_bytes, stream), "wal_validate")
+
+
+def wal_unpack_matrix(m, T, site_pos, site_sign, alpha, beta, U, V, stream):
+    return _check(lib.wal_unpack_matrix(ctypes.byref(m), T, site_pos, site_sign, alpha, beta, U, V,
+                                        stream), "wal_unpack_matrix")
+
+
+def wal_workspace_bytes(m, M):
+    return int(lib.wal_workspace_bytes(ctypes.byref(m), M))
+
+
+def wal_gemv(m, x, y, ws, ws_bytes, stream):
+    return _check(lib.wal_gemv(ctypes.byref(m), x, y, ws, ws_bytes, stream), "wal_gemv")
+
+
+def wal_gemm_small_m(m, X, M, ldx, Y, ldy, ws, ws_bytes, stream):
+    return _check(lib.wal_gemm_small_m(ctypes.byref(m), X, M, ldx, Y, ldy, ws, ws_bytes, stream),
+                  "wal_gemm_small_m")
+
+
+def wal_device_status(ws, stream):
+    return _check(lib.wal_device_status(ws, stream), "wal_device_status")
+
+
+def wal_body_workspace_bytes(mats, M):
+    arr = (wal_matrix * len(mats))(*mats)
+    return int(lib.wal_body_workspace_bytes(arr, len(mats), M))
+
+
+def wal_body_pass(plan, mats, stage_of, xs, ys, M, ws, ws_bytes, stream):
+    """plan: a ctypes.c_void_p holding the plan handle (None on the first call)."""
+    n = len(mats)
+    marr = (wal_matrix * n)(*mats)
+    sarr = (ctypes.c_int32 * n)(*stage_of)
+    xarr = (_vp * n)(*xs)
+    yarr = (_vp * n)(*ys)
+    return _check(lib.wal_body_pass(ctypes.byref(plan), marr, n, sarr, xarr, yarr, M, ws, ws_bytes,
+                                    stream), "wal_body_pass")
+
+
+def wal_body_plan_destroy(plan):
+    lib.wal_body_plan_destroy(plan)

@@ -1,0 +1,92 @@
+"""Device-resident packed matrices and the body-pass helper (argument marshalling only)."""
+import ctypes
+
+import numpy as np
+import torch
+
+from . import _abi
+from ._abi import wal_matrix
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    if isinstance(a, torch.Tensor):
+        return a.data_ptr()
+    return a.ctypes.data
+
+
+def pack_host(c):
+    """Pack dense components (attributes N, K, k, r, T, site_pos, site_sign, alpha,
+    beta, U, V, lr_scale as numpy arrays) with the library's host converter.
+    Returns the six layout-v1 buffers as numpy uint8 arrays."""
+    sizes = _abi.wal_packed_sizes(c.N, c.K, c.k, c.r)
+    out = [np.empty(s, dtype=np.uint8) for s in sizes]
+    arrs = [np.ascontiguousarray(c.T, np.int8),
+            np.ascontiguousarray(c.site_pos, np.uint8) if c.k else None,
+            np.ascontiguousarray(c.site_sign, np.int8) if c.k else None,
+            np.ascontiguousarray(c.alpha, np.uint16),
+            np.ascontiguousarray(c.beta, np.uint16) if c.k else None,
+            np.ascontiguousarray(c.U, np.int8) if c.r else None,
+            np.ascontiguousarray(c.V, np.int8) if c.r else None,
+            np.ascontiguousarray(c.lr_scale, np.uint16) if c.r else None]
+    _abi.wal_pack_matrix(*[_ptr(a) for a in arrs], c.N, c.K, c.k, c.r,
+                         [_ptr(o) if o.size else None for o in out])
+    return out
+
+
+class PackedMatrix:
+    """Six layout-v1 buffers on a CUDA device plus their wal_matrix descriptor."""
+
+    def __init__(self, bufs, N, K, k, r, device="cuda"):
+        self.N, self.K, self.k, self.r = N, K, k, r
+        self.bufs = [torch.from_numpy(np.ascontiguousarray(b).view(np.uint8).reshape(-1)).to(device)
+                     if np.size(b) else None for b in bufs]
+        self.desc = wal_matrix(N, K, k, r, *[_ptr(b) if b is not None else None for b in self.bufs])
+
+    @property
+    def nbytes(self):
+        return sum(b.numel() for b in self.bufs if b is not None)
+
+    def workspace_bytes(self, M=1):
+        return _abi.wal_workspace_bytes(self.desc, M)
+
+
+def to_device(bufs, N, K, k, r, device="cuda"):
+    return PackedMatrix(bufs, N, K, k, r, device)
+
+
+def _stream_handle(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+class BodyPass:
+    """Owns a wal_body_plan handle and its workspace; run() replays the graph."""
+
+    def __init__(self, mats, stage_of, xs, ys, M=1, device="cuda"):
+        self.mats = list(mats)
+        self.descs = [m.desc for m in self.mats]
+        self.stage_of = [int(s) for s in stage_of]
+        self.xs, self.ys, self.M = list(xs), list(ys), M
+        nb = _abi.wal_body_workspace_bytes(self.descs, M)
+        if nb == 0:
+            raise _abi.WalError(_abi.WAL_ERR_ARG, "wal_body_workspace_bytes")
+        self.ws = torch.empty(nb, dtype=torch.uint8, device=device)
+        self.plan = ctypes.c_void_p(None)
+
+    def run(self, stream=None):
+        _abi.wal_body_pass(self.plan, self.descs, self.stage_of, [x.data_ptr() for x in self.xs],
+                           [y.data_ptr() for y in self.ys], self.M, self.ws.data_ptr(), self.ws.numel(),
+                           _stream_handle(stream))
+
+    def close(self):
+        if self.plan.value:
+            _abi.wal_body_plan_destroy(self.plan)
+            self.plan = ctypes.c_void_p(None)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

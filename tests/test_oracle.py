@@ -46,8 +46,10 @@ def test_golden_codes_decode_by_hand():
     """Decode the fixture's hex bytes with the oracle and compare with the
     trits listed in the fixture."""
     c, _, _, codes_hex = load("codes_row16")
-    raw = np.frombuffer(codes_hex + bytes(0), dtype=np.uint8)
-    bufs = [raw, np.zeros(0, np.uint8), np.array([0x3C00], np.uint16),
+    raw = np.frombuffer(codes_hex, dtype=np.uint8)
+    scales = np.zeros(16, np.uint8)
+    scales[:2] = np.frombuffer(np.array([0x3C00], np.uint16).tobytes(), np.uint8)
+    bufs = [raw, np.zeros(0, np.uint8), scales,
             np.zeros(0, np.uint8), np.zeros(0, np.uint8), np.zeros(0, np.uint8)]
     u = oracle.unpack(bufs, 1, 128, 0, 0)
     assert np.array_equal(u.T, c.T)
@@ -179,7 +181,7 @@ def test_matmul_columns_equal_matvec(mid):
 def test_pq2_size_per_group():
     """T + alpha (k = 0, r = 0) costs 32 B of codes + 2 B of FP16 scale per
     128 weights = 34 B = 2.125 bit/weight (PQ2_0 on the WAL2-Ternary-27B card)."""
-    s = oracle.packed_sizes(1, 128, 0, 0)
+    s = oracle.payload_sizes(1, 128, 0, 0)
     assert s[0] == 32 and s[2] == 2 and sum(s) == 34
     assert oracle.bits_per_weight(4096, 4096, 0, 0) == 2.125
 
@@ -200,7 +202,7 @@ def test_unpack_rejects_reserved_code():
     c = gen_components(2, 128, 2, 1, config_id=80)
     bufs = oracle.pack(c)
     bufs[0] = bufs[0].copy()
-    bufs[0][1] |= np.uint32(3 << 6)
+    bufs[0][5] |= np.uint8(3 << 2)
     with pytest.raises(oracle.FormatError):
         oracle.unpack(bufs, 2, 128, 2, 1)
 
@@ -220,6 +222,20 @@ def test_unpack_rejects_wrong_size():
     bufs[2] = bufs[2][:-1]
     with pytest.raises(oracle.FormatError):
         oracle.unpack(bufs, 2, 128, 4, 0)
+
+
+def test_unpack_rejects_nonzero_padding():
+    c = gen_components(3, 128, 2, 0, config_id=80)   # 12 site bytes padded to 16
+    bufs = oracle.pack(c)
+    bufs[1] = bufs[1].copy()
+    bufs[1][-1] = 1
+    with pytest.raises(oracle.FormatError):
+        oracle.unpack(bufs, 3, 128, 2, 0)
+
+
+def test_padding_to_16_bytes():
+    assert oracle.packed_sizes(3, 128, 2, 1) == [96, 16, 16, 16, 16, 16]
+    assert oracle.payload_sizes(3, 128, 2, 1) == [96, 6, 12, 12, 16, 2]
 
 
 @pytest.mark.parametrize("shape", [(2, 100, 0, 0), (2, 128, 3, 0), (2, 128, 0, 33), (0, 128, 0, 0)])

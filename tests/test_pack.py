@@ -1,0 +1,90 @@
+"""Host converter (wal_pack_matrix) against the oracle's own packer, CPU only."""
+import numpy as np
+import pytest
+
+import oracle
+import ternary_sparse_binary_b200 as wal
+from wal_synth import Components, gen_components
+
+from golden_io import fixture_names, load
+
+
+SHAPES = [(512, 1024, 8, 4), (3, 128, 2, 1), (7, 256, 0, 0), (5, 384, 4, 32), (33, 2176, 8, 8),
+          (1, 128, 8, 0), (17, 640, 2, 31), (4, 4096, 0, 3)]
+
+
+@pytest.mark.parametrize("N,K,k,r", SHAPES)
+def test_pack_matches_oracle_bytes(N, K, k, r):
+    c = gen_components(N, K, k, r, config_id=81, matrix_index=N + K + k + r)
+    mine = wal.pack_host(c)
+    ref = oracle.pack(c)
+    assert [m.size for m in mine] == oracle.packed_sizes(N, K, k, r)
+    for i, (a, b) in enumerate(zip(mine, ref)):
+        assert np.array_equal(a, b), f"buffer {i} differs"
+
+
+@pytest.mark.parametrize("name", fixture_names())
+def test_pack_golden(name):
+    c, _, _, codes_hex = load(name)
+    mine = wal.pack_host(c)
+    assert all(np.array_equal(a, b) for a, b in zip(mine, oracle.pack(c)))
+    if codes_hex is not None:
+        assert mine[0][: len(codes_hex)].tobytes() == codes_hex
+
+
+def test_pack_roundtrip_through_oracle_decoder():
+    c = gen_components(64, 1024, 8, 16, config_id=82)
+    u = oracle.unpack(wal.pack_host(c), 64, 1024, 8, 16)
+    for f in ("T", "site_pos", "site_sign", "alpha", "beta", "U", "V", "lr_scale"):
+        assert np.array_equal(getattr(u, f), getattr(c, f)), f
+
+
+@pytest.mark.parametrize("shape", [(2, 100, 0, 0), (2, 128, 3, 0), (2, 128, 0, 33), (0, 128, 0, 0), (2, 0, 0, 0)])
+def test_sizes_reject_bad_shapes(shape):
+    with pytest.raises(wal.WalError) as e:
+        wal.wal_packed_sizes(*shape)
+    assert e.value.status == wal.WAL_ERR_SHAPE
+
+
+def _bad(mut):
+    c = gen_components(4, 256, 4, 2, config_id=83)
+    mut(c)
+    with pytest.raises(wal.WalError) as e:
+        wal.pack_host(c)
+    return e.value.status
+
+
+def test_pack_rejects_trit_out_of_range():
+    def m(c): c.T[1, 7] = 2
+    assert _bad(m) == wal.WAL_ERR_FORMAT
+
+
+def test_pack_rejects_duplicate_site():
+    def m(c): c.site_pos[2, 1, 1] = c.site_pos[2, 1, 0]
+    assert _bad(m) == wal.WAL_ERR_FORMAT
+
+
+def test_pack_rejects_unsorted_sites():
+    def m(c): c.site_pos[0, 0, :] = c.site_pos[0, 0, ::-1].copy()
+    assert _bad(m) == wal.WAL_ERR_FORMAT
+
+
+def test_pack_rejects_position_128():
+    def m(c): c.site_pos[0, 1, 3] = 128
+    assert _bad(m) == wal.WAL_ERR_FORMAT
+
+
+def test_pack_rejects_bad_sign_and_lowrank():
+    def m(c): c.site_sign[3, 0, 0] = 0
+    assert _bad(m) == wal.WAL_ERR_FORMAT
+
+    def m2(c): c.V[5, 1] = 0
+    assert _bad(m2) == wal.WAL_ERR_FORMAT
+
+
+def test_pack_rejects_null_buffers():
+    c = gen_components(4, 256, 4, 2, config_id=83)
+    with pytest.raises(wal.WalError) as e:
+        wal.wal_pack_matrix(c.T.ctypes.data, None, None, c.alpha.ctypes.data, None, None, None, None,
+                            4, 256, 4, 2, [None] * 6)
+    assert e.value.status == wal.WAL_ERR_ARG

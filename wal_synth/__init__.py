@@ -24,4 +24,7 @@ from .gen import (  # noqa: F401
     workload_id,
     WORKLOAD_IDS,
     CONFIG_SEED,
+    LAYER_8B,
+    LAYER_27B,
+    stream_seed,
 )
