@@ -4,18 +4,17 @@
 // README); here the graph holds the products of all body matrices in model
 // order, grouped into dependency stages.
 #include "wal_internal.h"
+#include "wal_stream.h"
 
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <vector>
 
 namespace wal {
-int launch_product_m1(const wal_matrix* m, const uint16_t* X, int M, int ldx, int m_index, float* y,
-                      void* ws, size_t ws_bytes, cudaStream_t stream, bool do_prep);
-size_t product_ws_bytes(const wal_matrix* m, int M);
 int check_product_args(const wal_matrix* m, const void* X, int M, int ldx, const void* Y, int ldy);
+StreamItem make_item(const wal_matrix* m, const uint16_t* x, float* y);
 }  // namespace wal
-
 using namespace wal;
 
 struct wal_body_plan {
@@ -55,19 +54,38 @@ void release(wal_body_plan* p) {
   p->graph = nullptr;
 }
 
-size_t per_matrix_ws(const wal_matrix& m, int M) { return align_up(product_ws_bytes(&m, M), 256); }
+// One launch of the capture: products that share K, all in one dependency stage.
+struct LaunchGroup {
+  int first, count;  // matrices [first, first + count)
+};
+
+std::vector<LaunchGroup> group_launches(const wal_matrix* mats, int n, const int32_t* stage_of, int M) {
+  std::vector<LaunchGroup> out;
+  const int per_launch = std::max(1, kMaxItems / M);
+  int i = 0;
+  while (i < n) {
+    int j = i + 1;
+    while (j < n && stage_of[j] == stage_of[i] && mats[j].K == mats[i].K && j - i < per_launch) ++j;
+    out.push_back({i, j - i});
+    i = j;
+  }
+  return out;
+}
+
+int add_prefetch(PrefetchRange* pf, int n_pf, const void* p, size_t bytes) {
+  if (!p || bytes == 0 || n_pf >= kMaxPrefetch) return n_pf;
+  pf[n_pf].ptr = p;
+  pf[n_pf].bytes = bytes & ~(size_t)15;
+  return pf[n_pf].bytes ? n_pf + 1 : n_pf;
+}
 
 }  // namespace
 
 extern "C" size_t wal_body_workspace_bytes(const wal_matrix* mats, int n_mats, int M) {
   if (!mats || n_mats <= 0 || M < 1) return 0;
-  size_t total = 0;
-  for (int i = 0; i < n_mats; ++i) {
-    size_t b = wal_workspace_bytes(&mats[i], M);
-    if (!b) return 0;
-    total += align_up(b, 256);
-  }
-  return total;
+  for (int i = 0; i < n_mats; ++i)
+    if (!wal_workspace_bytes(&mats[i], M)) return 0;
+  return 512;  // status header only: the batch-1 kernels keep every intermediate on chip
 }
 
 extern "C" int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n_mats, const int32_t* stage_of,
@@ -107,13 +125,33 @@ extern "C" int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n
     cudaError_t e = cudaStreamBeginCapture(p->capture_stream, cudaStreamCaptureModeThreadLocal);
     if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("begin capture: ") + cudaGetErrorString(e));
     int st = WAL_OK;
-    char* wsp = static_cast<char*>(ws);
-    for (int i = 0; i < n_mats && st == WAL_OK; ++i) {
-      const size_t b = per_matrix_ws(mats[i], M);
-      for (int mi = 0; mi < M && st == WAL_OK; ++mi)
-        st = launch_product_m1(&mats[i], xs[i], M, mats[i].K, mi, ys[i] + (size_t)mi * mats[i].N, wsp, b,
-                               p->capture_stream, mi == 0);
-      wsp += b;
+    const std::vector<LaunchGroup> groups = group_launches(mats, n_mats, stage_of, M);
+    for (size_t gi = 0; gi < groups.size() && st == WAL_OK; ++gi) {
+      const LaunchGroup& lg = groups[gi];
+      StreamParams prm = {};
+      prm.K = mats[lg.first].K;
+      prm.status = reinterpret_cast<int32_t*>(align_up((uintptr_t)ws, 256));
+      int n_items = 0;
+      for (int i = lg.first; i < lg.first + lg.count; ++i)
+        for (int mi = 0; mi < M; ++mi)
+          prm.items[n_items++] = make_item(&mats[i], xs[i] + (size_t)mi * mats[i].K, ys[i] + (size_t)mi * mats[i].N);
+      prm.n_items = n_items;
+      // warm L2 with the weights of the next launch
+      if (gi + 1 < groups.size()) {
+        const LaunchGroup& nx = groups[gi + 1];
+        int n_pf = 0;
+        for (int i = nx.first; i < nx.first + nx.count; ++i) {
+          size_t sz[6];
+          sizes_of(mats[i].N, mats[i].K, mats[i].k, mats[i].r, sz);
+          n_pf = add_prefetch(prm.pf, n_pf, mats[i].codes, sz[0]);
+          n_pf = add_prefetch(prm.pf, n_pf, mats[i].sites, sz[1]);
+          n_pf = add_prefetch(prm.pf, n_pf, mats[i].scales, sz[2]);
+        }
+        prm.n_pf = n_pf;
+      }
+      StreamLaunch L;
+      st = plan_stream(prm.items, n_items, prm.K, &L);
+      if (st == WAL_OK) st = launch_stream(prm, L, p->capture_stream, gi > 0);
     }
     cudaGraph_t g = nullptr;
     e = cudaStreamEndCapture(p->capture_stream, &g);

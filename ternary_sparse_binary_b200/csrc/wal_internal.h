@@ -10,9 +10,9 @@
 namespace wal {
 
 constexpr int kGroup = 128;        // weights per scale group
-constexpr int kMaxK = 65536;       // largest K handled by this build
-constexpr int kWordsPerLane = 4;   // 64 columns per lane in the decode-GEMV
-constexpr int kSliceCols = 32 * kWordsPerLane * 16;  // 2048 columns per K-slice (one warp)
+constexpr int kMaxK = 24576;       // largest K handled by this build
+constexpr int kWordsPerLane = 8;   // one 128-group (8 code words) per lane in the decode-GEMV
+constexpr int kSliceCols = 32 * kWordsPerLane * 16;  // 4096 columns per K-slice (one warp)
 constexpr int kLimbWords = 12;     // 3 limbs x 4 slots of uint32 per 16-column code word
 
 int fail(int status, const std::string& msg);
