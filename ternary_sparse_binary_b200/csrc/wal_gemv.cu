@@ -4,6 +4,7 @@
 #include "wal_internal.h"
 #include "wal_device.cuh"
 #include "wal_stream.h"
+#include "wal_tc.h"
 
 #include <algorithm>
 #include <mutex>
@@ -160,7 +161,7 @@ int launch_rows(const wal_matrix* m, const uint16_t* X, int ldx, float* Y, int l
 }
 
 size_t product_ws_bytes(const wal_matrix* m, int M) {
-  (void)m; (void)M;
+  if (M > kMaxItems) return tc_ws_bytes(m, M);
   return ws_layout(0, 0, 0, 0, 0).total;
 }
 
@@ -184,9 +185,9 @@ extern "C" size_t wal_workspace_bytes(const wal_matrix* m, int M) {
   return product_ws_bytes(m, M);
 }
 
-static int ws_check(void* ws, size_t ws_bytes) {
+static int ws_check(void* ws, size_t ws_bytes, size_t need) {
   if (!ws) return fail(WAL_ERR_ARG, "workspace is NULL");
-  if (ws_bytes < ws_layout(0, 0, 0, 0, 0).total) return fail(WAL_ERR_WORKSPACE, "workspace too small");
+  if (need == 0 || ws_bytes < need) return fail(WAL_ERR_WORKSPACE, "workspace too small");
   return WAL_OK;
 }
 
@@ -194,7 +195,7 @@ extern "C" int wal_gemv(const wal_matrix* m, const uint16_t* x, float* y, void* 
                         wal_stream_t stream) {
   int st = check_product_args(m, x, 1, m ? m->K : 0, y, m ? m->N : 0);
   if (st) return st;
-  st = ws_check(ws, ws_bytes);
+  st = ws_check(ws, ws_bytes, product_ws_bytes(m, 1));
   if (st) return st;
   return launch_rows(m, x, m->K, y, m->N, 0, 1, (cudaStream_t)stream, false, nullptr, 0,
                      reinterpret_cast<int32_t*>(ws_base(ws)));
@@ -204,8 +205,10 @@ extern "C" int wal_gemm_small_m(const wal_matrix* m, const uint16_t* X, int M, i
                                 void* ws, size_t ws_bytes, wal_stream_t stream) {
   int st = check_product_args(m, X, M, ldx, Y, ldy);
   if (st) return st;
-  st = ws_check(ws, ws_bytes);
+  st = ws_check(ws, ws_bytes, product_ws_bytes(m, M));
   if (st) return st;
+  // more than 16 activation rows: the product is a dense contraction (tensor cores)
+  if (M > kMaxItems) return launch_tc(m, X, M, ldx, Y, ldy, ws_base(ws), (cudaStream_t)stream);
   for (int m0 = 0; m0 < M; m0 += kMaxItems) {
     st = launch_rows(m, X, ldx, Y, ldy, m0, std::min(kMaxItems, M - m0), (cudaStream_t)stream, false, nullptr, 0,
                      reinterpret_cast<int32_t*>(ws_base(ws)));

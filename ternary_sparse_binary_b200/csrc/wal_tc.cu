@@ -1,0 +1,579 @@
+// Tensor-core product for batches of more than 16 activation rows
+//   Y[M][N] = X[M][K] W^T,   W = alpha*T + beta*R + U diag(s) V^T
+// (WAL-Ternary-8B model card, "Representation").  Only here is the product a
+// dense contraction, so only here do the 5th-generation tensor cores run.
+//
+// Exact FP16 operands.  alpha*t and beta*r (t, r in {-1, 0, +1}, alpha and beta
+// FP16) are FP16 values exactly, so W's ternary and residual planes are
+// decoded to FP16 with the group scales folded in: A_T = alpha (x) T and
+// A_R = beta (x) R, two MMAs into one FP32 accumulator in tensor memory (their
+// sum alpha*t + beta*r would not be exact in FP16 where a site falls on a
+// nonzero trit, so the planes stay apart).  X is BF16; scaled by a power of
+// two per activation row it is FP16 exactly (see tc_prep_kernel), and the
+// power of two comes off again in the epilogue.
+//
+// Launch 1, tc_prep_kernel (one CTA per activation row m):
+//   - 2^sc_m puts max|x_m| in [2^14, 2^15); x_m * 2^sc_m is written as FP16,
+//     exact for every element down to 2^-31 of the row maximum and rounded to
+//     nearest-even below that, into the pre-tiled B operand: per 64-column
+//     K-block and tile of activation rows, M_tile rows of 128 bytes in the
+//     tensor core's 128-byte-swizzled K-major layout, so one bulk copy moves a
+//     whole B tile.  Inside every 16 columns the order is the 4 x 4 transpose
+//     (column 16b + 4i + j goes to position 16b + 4j + i), which is the order
+//     the trit decode below produces.
+//   - WALB2 phase 1: z_r = sum_j V[j][r] x_j 2^sc_m in FP32 (fixed order), then
+//     2^t_m puts max_r |z_r| in [2^14, 2^15) and z_r 2^-t_m is split into an
+//     FP16 pair hi + lo (about 22 significant bits), stored as the B operand
+//     of one more MMA: columns 0..r-1 hi, r..2r-1 lo, zero to 64.
+// Launch 2, tc_kernel: one CTA per (128-row tile of W, tile of activation
+// rows), 10 warps:
+//   warp 0    lane 0 streams the B tiles (bulk copies, mbarrier ring);
+//   warp 1    allocates tensor memory; lane 0 issues the MMAs:
+//             D  += A_T B + A_R B          per 64-column K-block,
+//             D2  = A_lr B_lr              once, A_lr[n] = (+-s_r, +-s_r) from U;
+//   warps 2-9 decode: two teams of 128 threads, one output row per thread,
+//             team h taking the K-blocks 2g + h of every group g.  Per 16
+//             trits (one code word) four masks give the byte codes of slots
+//             {s, 4+s, 8+s, 12+s}; a multiply-add turns each code c into the
+//             byte-permute selector (2c, 2c+1), and byte permutes pick
+//             {-alpha, 0, +alpha} as FP16 pairs from two table registers.  The
+//             residual plane is zeroed and the k sites scattered as +-beta.
+//             Then the same warps run the epilogue:
+//             y[m][n] = (D + D2 2^t_m) 2^-sc_m.
+// All mbarrier waits are bounded; one that gives up records WAL_ERR_TIMEOUT in
+// the status word and its role stops issuing work.
+#include "wal_internal.h"
+#include "wal_device.cuh"
+#include "wal_ptx.cuh"
+#include "wal_tc.h"
+
+#include <algorithm>
+#include <mutex>
+
+namespace wal {
+
+using namespace ptx;
+
+namespace {
+
+constexpr int kRows = 128;           // MMA M: rows of W per tile
+constexpr int kBlockK = 64;          // K per pipeline stage: one 128-byte row of FP16
+constexpr int kMaxTileM = 256;       // MMA N limit
+constexpr int kThreads = 320;        // 10 warps
+constexpr int kPrepThreads = 256;
+constexpr uint32_t kATile = kRows * 128u;  // 16 KB: one FP16 plane of a stage
+constexpr int kMaxStages = 4;
+
+struct TcPrepParams {
+  const uint16_t* X;
+  int ldx, M, K, r, M_tile;
+  const uint32_t* vbits;
+  char* xt;      // [n_mt][K/64][M_tile x 128 B]
+  char* zt;      // [n_mt][M_tile x 128 B]
+  float2* scal;  // [M_pad] {2^-sc_m, 2^t_m}
+  int32_t* status;
+};
+
+struct TcParams {
+  const uint32_t* codes;
+  const uint8_t* sites;
+  const uint16_t* scales;
+  const uint32_t* ubits;
+  const uint16_t* lr;
+  const char* xt;
+  const char* zt;
+  const float2* scal;
+  float* Y;
+  int ldy, N, K, r, M, M_tile, stages, n_tiles_n;
+  uint32_t d2_col;     // tensor-memory column of D2
+  uint32_t tmem_cols;  // allocated tensor-memory columns
+  int32_t* status;
+};
+
+// 2^e as a double, e in [-1022, 1023].
+__device__ __forceinline__ double pow2d(int e) { return __longlong_as_double((long long)(e + 1023) << 52); }
+
+// floor(log2(v)) of a finite nonzero float bit pattern (sign ignored).
+__device__ __forceinline__ int ilog2f_bits(uint32_t b) {
+  const uint32_t ex = (b >> 23) & 0xFFu;
+  if (ex) return (int)ex - 127;
+  return -149 + (31 - __clz((int)(b & 0x7FFFFFu)));
+}
+
+// ---------------------------------------------------------------------------
+// launch 1: FP16 image of X (pre-tiled B operand) and WALB2 phase 1
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kPrepThreads) tc_prep_kernel(const TcPrepParams p) {
+  const int m = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (m == 0 && tid == 0 && p.status) *p.status = 0;
+  const bool live = m < p.M;
+  const int KB = p.K / kBlockK, n16 = p.K / 16;
+  const int mt = m / p.M_tile, row = m % p.M_tile;
+  const uint16_t* xrow = p.X + (size_t)(live ? m : 0) * p.ldx;
+  __shared__ uint32_t s_red[kPrepThreads / 32];
+  __shared__ float s_z[kPrepThreads / 32][WAL_MAX_RANK];
+  __shared__ float s_zr[WAL_MAX_RANK];
+  __shared__ int s_t;
+
+  // largest |x| as a bit pattern (monotonic for finite values)
+  uint32_t mx = 0;
+  if (live)
+    for (int c = tid; c < p.K / 8; c += kPrepThreads) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(xrow) + c);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) mx = max(mx, max(w[q] & 0x7FFFu, (w[q] >> 16) & 0x7FFFu));
+    }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (lane == 0) s_red[warp] = mx;
+  __syncthreads();
+  mx = 0;
+#pragma unroll
+  for (int w = 0; w < kPrepThreads / 32; ++w) mx = max(mx, s_red[w]);
+  const int sc = mx ? 14 - ilog2f_bits(mx << 16) : 0;
+  const double f = pow2d(sc);
+
+  float acc[WAL_MAX_RANK];
+#pragma unroll
+  for (int q = 0; q < WAL_MAX_RANK; ++q) acc[q] = 0.f;
+  for (int b = tid; b < n16; b += kPrepThreads) {
+    float xs[16];
+    if (live) {
+      const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(xrow) + 2 * b);
+      const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(xrow) + 2 * b + 1);
+      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        xs[j] = (float)((double)dev::bf16_bits_to_float((w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu) * f);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) xs[j] = 0.f;
+    }
+    // FP16, 4 x 4 transposed inside the 16 columns
+    uint32_t hw[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int i0 = 2 * i, i1 = 2 * i + 1;
+      const int j0 = 4 * (i0 & 3) + (i0 >> 2), j1 = 4 * (i1 & 3) + (i1 >> 2);
+      hw[i] = (uint32_t)__half_as_ushort(__float2half_rn(xs[j0])) |
+              ((uint32_t)__half_as_ushort(__float2half_rn(xs[j1])) << 16);
+    }
+    const int kb = b >> 2, bq = b & 3;
+    char* tile = p.xt + ((size_t)mt * KB + kb) * ((size_t)p.M_tile * 128u);
+    *reinterpret_cast<uint4*>(tile + sw128((uint32_t)row, 2u * bq)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(tile + sw128((uint32_t)row, 2u * bq + 1u)) = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+    // WALB2 phase 1 partials: sum_j V[j][rho] x_j, V = -1 where the bit is set
+    if (p.r > 0) {
+#pragma unroll
+      for (int q = 0; q < WAL_MAX_RANK; ++q) {
+        if (q < p.r) {
+          const uint32_t bits = (__ldg(p.vbits + (size_t)q * (p.K / 32) + (b >> 1)) >> (16 * (b & 1))) & 0xFFFFu;
+          float s = 0.f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) s += __uint_as_float(__float_as_uint(xs[j]) ^ (((bits >> j) & 1u) << 31));
+          acc[q] += s;
+        }
+      }
+    }
+  }
+  if (tid == 0) p.scal[m] = make_float2((float)pow2d(-sc), 1.f);
+  if (p.r == 0) return;
+
+#pragma unroll
+  for (int q = 0; q < WAL_MAX_RANK; ++q) {
+    float v = acc[q];
+#pragma unroll
+    for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (lane == 0) s_z[warp][q] = v;
+  }
+  __syncthreads();
+  if (tid < 32) {
+    float z = 0.f;
+    if (tid < p.r)
+#pragma unroll
+      for (int w = 0; w < kPrepThreads / 32; ++w) z += s_z[w][tid];
+    s_zr[tid] = z;
+    uint32_t zm = __float_as_uint(z) & 0x7FFFFFFFu;
+#pragma unroll
+    for (int off = 16; off; off >>= 1) zm = max(zm, __shfl_xor_sync(0xffffffffu, zm, off));
+    if (tid == 0) {
+      int t = zm ? ilog2f_bits(zm) - 14 : 0;
+      t = max(-120, min(t, 120));
+      s_t = t;
+      p.scal[m] = make_float2((float)pow2d(-sc), (float)pow2d(t));
+    }
+  }
+  __syncthreads();
+  if (tid < 64) {
+    // column kk of the WALB2 B operand: hi of rank kk, lo of rank kk - r, else 0
+    float hv = 0.f;
+    if (live && tid < 2 * p.r) {
+      const int q = tid < p.r ? tid : tid - p.r;
+      const float v = (float)((double)s_zr[q] * pow2d(-s_t));
+      const float hi = __half2float(__float2half_rn(v));
+      hv = tid < p.r ? hi : __half2float(__float2half_rn(v - hi));
+    }
+    char* tile = p.zt + (size_t)mt * ((size_t)p.M_tile * 128u);
+    *reinterpret_cast<__half*>(tile + sw128((uint32_t)row, (uint32_t)tid >> 3) + 2 * (tid & 7)) = __float2half_rn(hv);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// launch 2: decode + tcgen05 MMA + epilogue
+// ---------------------------------------------------------------------------
+
+// 16 trits (one code word) -> two 16-byte chunks of FP16 {-a, 0, +a} in the
+// 4 x 4 transposed order.  ta = (-a, 0), tb = (+a, 0) as FP16 pairs; code c
+// selects bytes 2c, 2c+1 of (ta, tb).
+__device__ __forceinline__ void decode_word(uint32_t w, uint32_t ta, uint32_t tb, uint4& c0, uint4& c1) {
+  const uint32_t s0 = (w & 0x03030303u) * 0x22u + 0x10101010u;
+  const uint32_t s1 = ((w >> 2) & 0x03030303u) * 0x22u + 0x10101010u;
+  const uint32_t s2 = ((w >> 4) & 0x03030303u) * 0x22u + 0x10101010u;
+  const uint32_t s3 = ((w >> 6) & 0x03030303u) * 0x22u + 0x10101010u;
+  c0.x = __byte_perm(ta, tb, s0);        // trits 0, 4
+  c0.y = __byte_perm(ta, tb, s0 >> 16);  // 8, 12
+  c0.z = __byte_perm(ta, tb, s1);        // 1, 5
+  c0.w = __byte_perm(ta, tb, s1 >> 16);  // 9, 13
+  c1.x = __byte_perm(ta, tb, s2);        // 2, 6
+  c1.y = __byte_perm(ta, tb, s2 >> 16);  // 10, 14
+  c1.z = __byte_perm(ta, tb, s3);        // 3, 7
+  c1.w = __byte_perm(ta, tb, s3 >> 16);  // 11, 15
+}
+
+template <int KS>
+struct GroupLoad {
+  uint4 codes;
+  uint32_t sites_lo, sites_hi;
+  uint32_t scales;
+};
+
+template <int KS>
+__device__ __forceinline__ GroupLoad<KS> load_group(const TcParams& p, int n, int g, int h, int G) {
+  GroupLoad<KS> v;
+  const size_t rg = (size_t)n * G + g;
+  v.codes = __ldg(reinterpret_cast<const uint4*>(p.codes + (size_t)n * (p.K / 16) + 8 * g + 4 * h));
+  v.sites_lo = v.sites_hi = 0u;
+  if (KS == 8) {
+    const uint2 s = __ldg(reinterpret_cast<const uint2*>(p.sites + rg * 8));
+    v.sites_lo = s.x; v.sites_hi = s.y;
+  } else if (KS == 4) {
+    v.sites_lo = __ldg(reinterpret_cast<const uint32_t*>(p.sites + rg * 4));
+  } else if (KS == 2) {
+    v.sites_lo = __ldg(reinterpret_cast<const uint16_t*>(p.sites + rg * 2));
+  }
+  v.scales = KS ? __ldg(reinterpret_cast<const uint32_t*>(p.scales) + rg) : (uint32_t)__ldg(p.scales + rg);
+  return v;
+}
+
+template <int KS>
+__global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  constexpr bool kHasR = KS > 0;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t b_bytes = (uint32_t)p.M_tile * 128u;
+  const uint32_t stage_bytes = kATile * (kHasR ? 2u : 1u) + b_bytes;
+  const int S = p.stages;
+  const uint32_t bars = base + (uint32_t)S * stage_bytes;
+  // barriers: b_full[S], a_full[S], empty[S], acc_full
+  auto b_full = [&](int s) { return bars + 8u * s; };
+  auto a_full = [&](int s) { return bars + 8u * (S + s); };
+  auto empty = [&](int s) { return bars + 8u * (2 * S + s); };
+  const uint32_t acc_full = bars + 8u * (3 * S);
+  const uint32_t tmem_slot = acc_full + 8u;
+  const uint32_t scal_s = (tmem_slot + 4u + 15u) & ~15u;
+  auto a_t = [&](int s) { return base + (uint32_t)s * stage_bytes; };
+  auto a_r = [&](int s) { return base + (uint32_t)s * stage_bytes + kATile; };
+  auto b_t = [&](int s) { return base + (uint32_t)s * stage_bytes + kATile * (kHasR ? 2u : 1u); };
+
+  const int n_tile = blockIdx.x % p.n_tiles_n, mt = blockIdx.x / p.n_tiles_n;
+  const int G = p.K / 128, KB = p.K / kBlockK;
+  const bool has_lr = p.r > 0;
+  const int n_iter = KB + (has_lr ? 1 : 0);
+  const uint32_t ncols = p.tmem_cols;
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(b_full(s), 1);
+      mbar_init(a_full(s), 128);
+      mbar_init(empty(s), 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init_fence();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = lds32(tmem_slot);
+
+  if (warp == 0) {
+    // ---- B producer ----
+    if (lane == 0) {
+      for (int i = 0; i < n_iter; ++i) {
+        const int s = i % S;
+        const uint32_t ph = (uint32_t)(i / S) & 1u;
+        if (!mbar_wait(empty(s), ph ^ 1u, p.status)) break;
+        const char* src = i < KB ? p.xt + ((size_t)mt * KB + i) * b_bytes : p.zt + (size_t)mt * b_bytes;
+        mbar_arrive_expect_tx(b_full(s), b_bytes);
+        bulk_g2s(b_t(s), src, b_bytes, b_full(s));
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_f32(kRows, (uint32_t)p.M_tile);
+      bool ok = true;
+      for (int i = 0; i < KB && ok; ++i) {
+        const int s = i % S;
+        const uint32_t ph = (uint32_t)(i / S) & 1u;
+        ok = mbar_wait(b_full(s), ph, p.status) && mbar_wait(a_full(s), ph, p.status);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBlockK / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128(b_t(s) + 32u * kk);
+          mma_f16(tmem, sdesc_sw128(a_t(s) + 32u * kk), bd, idesc, (i | kk) != 0);
+          if (kHasR) mma_f16(tmem, sdesc_sw128(a_r(s) + 32u * kk), bd, idesc, 1u);
+        }
+        mma_commit(empty(s));
+      }
+      if (ok && has_lr) {
+        const int s = KB % S;
+        const uint32_t ph = (uint32_t)(KB / S) & 1u;
+        ok = mbar_wait(b_full(s), ph, p.status) && mbar_wait(a_full(s), ph, p.status);
+        if (ok) {
+          tc_fence_after();
+          for (int kk = 0; kk < (2 * p.r + 15) / 16; ++kk)
+            mma_f16(tmem + p.d2_col, sdesc_sw128(a_t(s) + 32u * kk), sdesc_sw128(b_t(s) + 32u * kk), idesc,
+                    kk != 0);
+          mma_commit(empty(s));
+        }
+      }
+      mma_commit(acc_full);
+    }
+  } else {
+    // ---- decoders, then epilogue ----
+    const int h = (warp - 2) >> 2;      // team
+    const int q = warp & 3;             // tensor-memory lane quarter
+    const int row = 32 * q + lane;
+    const int n = n_tile * kRows + row;
+    const bool live = n < p.N;
+    const uint32_t rowoff = (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u;
+    const uint32_t r7 = (uint32_t)row & 7u;
+    bool ok = true;
+
+    GroupLoad<KS> cur = {}, nxt = {};
+    if (live) cur = load_group<KS>(p, n, 0, h, G);
+    if (live && G > 1) nxt = load_group<KS>(p, n, 1, h, G);
+    for (int g = 0; g < G && ok; ++g) {
+      GroupLoad<KS> nn = {};
+      if (live && g + 2 < G) nn = load_group<KS>(p, n, g + 2, h, G);
+      const int i = 2 * g + h, s = i % S;
+      const uint32_t ph = (uint32_t)(i / S) & 1u;
+      ok = mbar_wait(empty(s), ph ^ 1u, p.status);
+      if (!ok) break;
+      const uint32_t at = a_t(s) + rowoff;
+      // ternary plane: alpha (x) T
+      const uint32_t alpha = cur.scales & 0xFFFFu;
+      const uint32_t ta = live ? (alpha ^ 0x8000u) : 0u, tb = alpha;
+      const uint32_t cw[4] = {cur.codes.x, cur.codes.y, cur.codes.z, cur.codes.w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint4 c0, c1;
+        decode_word(cw[w], ta, tb, c0, c1);
+        sts128(at + ((((uint32_t)(2 * w)) ^ r7) << 4), c0);
+        sts128(at + ((((uint32_t)(2 * w + 1)) ^ r7) << 4), c1);
+      }
+      if (kHasR) {
+        // residual plane: zero the row, scatter +-beta at this half's sites
+        const uint32_t ar = a_r(s) + rowoff;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) sts128(ar + (((uint32_t)c ^ r7) << 4), make_uint4(0u, 0u, 0u, 0u));
+        const uint32_t beta = cur.scales >> 16;
+#pragma unroll
+        for (int j = 0; j < KS; ++j) {
+          const uint32_t b = ((j < 4 ? cur.sites_lo : cur.sites_hi) >> (8 * (j & 3))) & 0xFFu;
+          if (live && ((b >> 6) & 1u) == (uint32_t)h) {
+            const uint32_t pos = b & 63u, jj = pos & 15u;
+            const uint32_t col = (pos & 48u) | ((jj & 3u) << 2) | (jj >> 2);
+            sts16(ar + ((((col >> 3) ^ r7) & 7u) << 4) + 2u * (col & 7u), beta ^ ((b & 0x80u) << 8));
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(a_full(s));
+      cur = nxt;
+      nxt = nn;
+    }
+    // WALB2 phase-2 operand A_lr[n] = (+-s_0 .. +-s_{r-1}, +-s_0 .. +-s_{r-1}, 0 ...)
+    if (ok && has_lr && h == (KB & 1)) {
+      const int s = KB % S;
+      const uint32_t ph = (uint32_t)(KB / S) & 1u;
+      ok = mbar_wait(empty(s), ph ^ 1u, p.status);
+      if (ok) {
+        const uint32_t u = live ? __ldg(p.ubits + (size_t)n * ((p.r + 31) / 32)) : 0u;
+        const uint32_t at = a_t(s) + rowoff;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t hw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint32_t v2 = 0u;
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) {
+              const int kk = 8 * c + 2 * e + hlf;
+              const int rho = kk < p.r ? kk : kk - p.r;
+              uint32_t v = 0u;
+              if (live && kk < 2 * p.r) v = (uint32_t)__ldg(p.lr + rho) ^ (((u >> rho) & 1u) << 15);
+              v2 |= v << (16 * hlf);
+            }
+            hw[e] = v2;
+          }
+          sts128(at + (((uint32_t)c ^ r7) << 4), make_uint4(hw[0], hw[1], hw[2], hw[3]));
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(a_full(s));
+      }
+    }
+
+    // ---- epilogue ----
+    for (int j = tid - 64; j < p.M_tile; j += 256) {
+      const int m = mt * p.M_tile + j;
+      const float2 v = m < p.M ? p.scal[m] : make_float2(0.f, 0.f);
+      sts64(scal_s + 8u * j, make_uint2(__float_as_uint(v.x), __float_as_uint(v.y)));
+    }
+    named_bar_sync(1, 256);
+    if (mbar_wait(acc_full, 0u, p.status)) {
+      tc_fence_after();
+      const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+      for (int c16 = h; c16 < p.M_tile / 16; c16 += 2) {
+        uint32_t d[16], e[16];
+        tmem_ld16(lane_base + 16u * c16, d);
+        if (has_lr) tmem_ld16(lane_base + p.d2_col + 16u * c16, e);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int col = 16 * c16 + j, m = mt * p.M_tile + col;
+          const uint2 sv = lds64(scal_s + 8u * col);
+          float y = __uint_as_float(d[j]);
+          if (has_lr) y = fmaf(__uint_as_float(e[j]), __uint_as_float(sv.y), y);
+          y *= __uint_as_float(sv.x);
+          if (live && m < p.M) p.Y[(size_t)m * p.ldy + n] = y;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, ncols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+std::once_flag g_tc_once;
+cudaError_t g_tc_err = cudaSuccess;
+int g_tc_smem_limit = 0;
+
+int tc_init() {
+  std::call_once(g_tc_once, [] {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&g_tc_smem_limit, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_tc_smem_limit);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_tc_smem_limit);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_tc_smem_limit);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_tc_smem_limit);
+    g_tc_err = e;
+  });
+  if (g_tc_err != cudaSuccess)
+    return fail(WAL_ERR_CUDA, std::string("tensor-core path initialisation: ") + cudaGetErrorString(g_tc_err));
+  return WAL_OK;
+}
+
+uint32_t pow2_ceil(uint32_t v) {
+  uint32_t p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+}  // namespace
+
+int plan_tc(const wal_matrix* m, int M, TcPlan* out) {
+  TcPlan P = {};
+  P.n_tiles_n = (m->N + kRows - 1) / kRows;
+  P.n_mt = (M + kMaxTileM - 1) / kMaxTileM;
+  P.M_tile = ((M + P.n_mt - 1) / P.n_mt + 15) / 16 * 16;
+  P.M_pad = P.n_mt * P.M_tile;
+  const uint32_t b_bytes = (uint32_t)P.M_tile * 128u;
+  const uint32_t stage_bytes = kATile * (m->k > 0 ? 2u : 1u) + b_bytes;
+  const uint32_t extra = 1024u /*alignment*/ + 8u * (3 * kMaxStages + 1) + 16u + 8u * kMaxTileM;
+  const uint32_t limit = g_tc_smem_limit > 0 ? (uint32_t)g_tc_smem_limit : 232448u;
+  P.stages = (int)std::min<uint32_t>(kMaxStages, (limit - extra) / stage_bytes);
+  if (P.stages < 2) return fail(WAL_ERR_UNSUPPORTED, "tensor-core tile does not fit in shared memory");
+  P.smem = extra + (uint32_t)P.stages * stage_bytes;
+  const uint32_t d2 = pow2_ceil((uint32_t)P.M_tile);
+  P.tmem_cols = std::max(32u, d2 * (m->r > 0 ? 2u : 1u));
+  P.off_scal = 0;
+  P.off_zt = align_up(256 + (size_t)P.M_pad * 8, 1024);
+  P.off_xt = align_up(P.off_zt + (m->r > 0 ? (size_t)P.n_mt * b_bytes : 0), 1024);
+  P.total = P.off_xt + (size_t)P.M_pad * m->K * 2;
+  *out = P;
+  return WAL_OK;
+}
+
+size_t tc_ws_bytes(const wal_matrix* m, int M) {
+  TcPlan P;
+  if (plan_tc(m, M, &P) != WAL_OK) return 0;
+  return 256 /*alignment slack*/ + 256 /*header*/ + P.total;
+}
+
+int launch_tc(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, int ldy, char* ws,
+              cudaStream_t stream) {
+  int st = tc_init();
+  if (st) return st;
+  TcPlan P;
+  st = plan_tc(m, M, &P);
+  if (st) return st;
+  int32_t* status = reinterpret_cast<int32_t*>(ws);
+  char* data = ws + 256;  // header occupies the first 256 bytes
+  TcPrepParams pp;
+  pp.X = X; pp.ldx = ldx; pp.M = M; pp.K = m->K; pp.r = m->r; pp.M_tile = P.M_tile;
+  pp.vbits = m->v_bits;
+  pp.xt = data + P.off_xt;
+  pp.zt = data + P.off_zt;
+  pp.scal = reinterpret_cast<float2*>(data + P.off_scal);
+  pp.status = status;
+  tc_prep_kernel<<<P.M_pad, kPrepThreads, 0, stream>>>(pp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("tc_prep_kernel launch: ") + cudaGetErrorString(e));
+
+  TcParams tp;
+  tp.codes = m->codes; tp.sites = m->sites; tp.scales = m->scales; tp.ubits = m->u_bits; tp.lr = m->lr_scale;
+  tp.xt = pp.xt; tp.zt = pp.zt; tp.scal = pp.scal;
+  tp.Y = Y; tp.ldy = ldy; tp.N = m->N; tp.K = m->K; tp.r = m->r; tp.M = M; tp.M_tile = P.M_tile;
+  tp.stages = P.stages; tp.n_tiles_n = P.n_tiles_n;
+  tp.d2_col = m->r > 0 ? P.tmem_cols / 2 : P.tmem_cols;
+  tp.tmem_cols = P.tmem_cols;
+  tp.status = status;
+  const dim3 grid(P.n_tiles_n * P.n_mt);
+  switch (m->k) {
+    case 0: tc_kernel<0><<<grid, kThreads, P.smem, stream>>>(tp); break;
+    case 2: tc_kernel<2><<<grid, kThreads, P.smem, stream>>>(tp); break;
+    case 4: tc_kernel<4><<<grid, kThreads, P.smem, stream>>>(tp); break;
+    default: tc_kernel<8><<<grid, kThreads, P.smem, stream>>>(tp); break;
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("tc_kernel launch: ") + cudaGetErrorString(e));
+  return WAL_OK;
+}
+
+}  // namespace wal

@@ -1,0 +1,32 @@
+// Tensor-core product for larger batches (see wal_tc.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/wal.h"
+
+namespace wal {
+
+// Geometry of one tensor-core call.
+struct TcPlan {
+  int n_tiles_n;  // 128-row tiles of W
+  int n_mt;       // activation tiles
+  int M_tile;     // activation rows per tile (MMA N), multiple of 16, <= 256
+  int M_pad;      // n_mt * M_tile
+  int stages;     // pipeline depth
+  uint32_t smem;  // dynamic shared memory per CTA
+  uint32_t tmem_cols;
+  // workspace offsets from the 256-byte aligned base
+  size_t off_scal, off_zt, off_xt, total;
+};
+
+int plan_tc(const wal_matrix* m, int M, TcPlan* out);
+// Scratch bytes of the tensor-core path (including the 256-byte alignment slack).
+size_t tc_ws_bytes(const wal_matrix* m, int M);
+int launch_tc(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, int ldy, char* ws_base,
+              cudaStream_t stream);
+
+}  // namespace wal

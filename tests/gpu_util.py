@@ -44,6 +44,7 @@ def run_gemm(pm, X_dev, M):
     ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
     w.wal_gemm_small_m(pm.desc, X_dev.data_ptr(), M, pm.K, Y.data_ptr(), pm.N, ws.data_ptr(), nb, stream())
     torch.cuda.synchronize()
+    w.wal_device_status(ws.data_ptr(), stream())
     return Y.cpu().numpy().astype(np.float64)
 
 
