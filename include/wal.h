@@ -133,6 +133,21 @@ int wal_gemv(const wal_matrix* m, const uint16_t* x, float* y, void* ws, size_t 
 int wal_gemm_small_m(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, int ldy,
                      void* ws, size_t ws_bytes, wal_stream_t stream);
 
+/* Y[M][ldy] = X[M][ldx] W^T on the tensor-core path (M >= 17) without a
+ * workspace argument.  The model cards have no counterpart to this entry
+ * point: it exists for callers that cannot hand the library scratch memory.
+ * Its scratch is a fixed array of WAL_NOALLOC_SCRATCH_BYTES in the library's
+ * own device memory (one per device, located once per device); a call whose
+ * scratch need, wal_workspace_bytes(m, M), is larger returns
+ * WAL_ERR_WORKSPACE, and M <= 16 returns WAL_ERR_SHAPE.  Nothing is
+ * allocated.  Every call on a device uses the same array, so calls that
+ * overlap in time on one device (other streams, other host threads) race on
+ * it: the caller must order them.  Asynchronous on `stream`; a bounded
+ * device wait that gives up is not reported by this entry point. */
+#define WAL_NOALLOC_SCRATCH_BYTES (16u << 20)
+int wal_gemm_tc_noalloc(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, int ldy,
+                        wal_stream_t stream);
+
 /* Read and clear the device status word in a workspace header (synchronises
  * `stream`).  Every product call clears the word when it starts, so it reports
  * on the last call that used this workspace.  WAL_OK or WAL_ERR_TIMEOUT. */

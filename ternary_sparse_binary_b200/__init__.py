@@ -7,10 +7,10 @@ cannot be loaded, importing this package raises.
 """
 from ._abi import (  # noqa: F401
     WAL_OK, WAL_ERR_ARG, WAL_ERR_SHAPE, WAL_ERR_FORMAT, WAL_ERR_WORKSPACE, WAL_ERR_CUDA,
-    WAL_ERR_UNSUPPORTED, WAL_ERR_TIMEOUT, WAL_MAX_RANK, WAL_MAX_SMALL_M,
+    WAL_ERR_UNSUPPORTED, WAL_ERR_TIMEOUT, WAL_MAX_RANK, WAL_MAX_SMALL_M, WAL_NOALLOC_SCRATCH_BYTES,
     WalError, wal_matrix, lib, lib_path, EXPORTED_SYMBOLS,
     wal_packed_sizes, wal_pack_matrix, wal_validate, wal_unpack_matrix, wal_workspace_bytes,
-    wal_gemv, wal_gemm_small_m, wal_device_status, wal_body_workspace_bytes, wal_body_pass,
+    wal_gemv, wal_gemm_small_m, wal_gemm_tc_noalloc, wal_device_status, wal_body_workspace_bytes, wal_body_pass,
     wal_body_plan_destroy, wal_status_string, wal_last_error,
 )
 from .packed import PackedMatrix, pack_host, to_device, BodyPass  # noqa: F401

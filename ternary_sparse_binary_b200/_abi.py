@@ -19,10 +19,11 @@ WAL_ERR_UNSUPPORTED = -6
 WAL_ERR_TIMEOUT = -7
 WAL_MAX_RANK = 32
 WAL_MAX_SMALL_M = 16
+WAL_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 EXPORTED_SYMBOLS = [
     "wal_packed_sizes", "wal_pack_matrix", "wal_validate", "wal_unpack_matrix",
-    "wal_workspace_bytes", "wal_gemv", "wal_gemm_small_m", "wal_device_status",
+    "wal_workspace_bytes", "wal_gemv", "wal_gemm_small_m", "wal_gemm_tc_noalloc", "wal_device_status",
     "wal_body_workspace_bytes", "wal_body_pass", "wal_body_plan_destroy",
     "wal_status_string", "wal_last_error",
 ]
@@ -61,6 +62,7 @@ lib.wal_workspace_bytes.argtypes = [_MP, _i]
 lib.wal_workspace_bytes.restype = _sz
 lib.wal_gemv.argtypes = [_MP, _vp, _vp, _vp, _sz, _vp]
 lib.wal_gemm_small_m.argtypes = [_MP, _vp, _i, _i, _vp, _i, _vp, _sz, _vp]
+lib.wal_gemm_tc_noalloc.argtypes = [_MP, _vp, _i, _i, _vp, _i, _vp]
 lib.wal_device_status.argtypes = [_vp, _vp]
 lib.wal_body_workspace_bytes.argtypes = [_MP, _i, _i]
 lib.wal_body_workspace_bytes.restype = _sz
@@ -120,6 +122,10 @@ def wal_gemv(m, x, y, ws, ws_bytes, stream):
 def wal_gemm_small_m(m, X, M, ldx, Y, ldy, ws, ws_bytes, stream):
     return _check(lib.wal_gemm_small_m(ctypes.byref(m), X, M, ldx, Y, ldy, ws, ws_bytes, stream),
                   "wal_gemm_small_m")
+
+
+def wal_gemm_tc_noalloc(m, X, M, ldx, Y, ldy, stream):
+    return _check(lib.wal_gemm_tc_noalloc(ctypes.byref(m), X, M, ldx, Y, ldy, stream), "wal_gemm_tc_noalloc")
 
 
 def wal_device_status(ws, stream):
