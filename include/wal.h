@@ -159,10 +159,15 @@ int wal_device_status(void* ws, wal_stream_t stream);
  * starts only after every product of stage s has finished (a matrix of a
  * later stage may read an output of an earlier one).  Stages must be
  * non-decreasing along the array.  mats, stage_of, xs and ys are host arrays
- * (of device pointers).
- * The first call builds *plan (a CUDA graph of the pass on `stream`); later
- * calls with identical arguments replay it.  A call whose arguments differ
- * from the plan's rebuilds it. */
+ * (of device pointers).  1 <= M <= 16.
+ * The first call builds *plan: launch tables (kept in ws) and a CUDA graph of
+ * the pass on `stream` (a header clear plus one persistent cooperative launch
+ * with a grid barrier between stages).  Later calls with identical arguments
+ * replay it; a call whose arguments differ rebuilds it (synchronising
+ * `stream` first).  ws belongs to the plan while the plan is in use: nothing
+ * else may write it between calls.  wal_body_workspace_bytes gives its size.
+ * A bounded wait that gives up records WAL_ERR_TIMEOUT in the ws header
+ * (wal_device_status). */
 typedef struct wal_body_plan wal_body_plan;
 size_t wal_body_workspace_bytes(const wal_matrix* mats, int n_mats, int M);
 int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n_mats,

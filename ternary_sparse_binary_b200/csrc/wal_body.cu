@@ -2,7 +2,9 @@
 // one CUDA graph on one GPU.  The WAL-Ternary-8B runtime executes its decode
 // step as a CUDA graph ("CUDA V18 Graph" in the speed table of the Kazakh
 // README); here the graph holds the products of all body matrices in model
-// order, grouped into dependency stages.
+// order, grouped into dependency stages, as one persistent cooperative
+// launch of the decode-GEMV kernel (groups of one stage back to back, a grid
+// barrier between stages).
 #include "wal_internal.h"
 #include "wal_stream.h"
 
@@ -54,7 +56,7 @@ void release(wal_body_plan* p) {
   p->graph = nullptr;
 }
 
-// One launch of the capture: products that share K, all in one dependency stage.
+// One group of the launch: products that share K, all in one dependency stage.
 struct LaunchGroup {
   int first, count;  // matrices [first, first + count)
 };
@@ -72,11 +74,16 @@ std::vector<LaunchGroup> group_launches(const wal_matrix* mats, int n, const int
   return out;
 }
 
-int add_prefetch(PrefetchRange* pf, int n_pf, const void* p, size_t bytes) {
-  if (!p || bytes == 0 || n_pf >= kMaxPrefetch) return n_pf;
-  pf[n_pf].ptr = p;
-  pf[n_pf].bytes = bytes & ~(size_t)15;
-  return pf[n_pf].bytes ? n_pf + 1 : n_pf;
+// Workspace of a body pass (offsets from the 256-byte aligned base):
+// [0, 256) header: status word at 0, grid-barrier counter at 128;
+// then the item table and the per-CTA schedules ([CTA][group] tile records)
+// the persistent launch reads.  There are at most n_mats groups.
+constexpr size_t kBarrierOffset = 128;
+constexpr int kMaxCtas = 1024;
+size_t items_offset() { return 256; }
+size_t sched_offset(int n_mats, int M) { return align_up(256 + (size_t)n_mats * M * sizeof(StreamItem), 256); }
+size_t body_ws_total(int n_mats, int M) {
+  return 256 /*alignment slack*/ + sched_offset(n_mats, M) + (size_t)kMaxCtas * n_mats * sizeof(TileRec);
 }
 
 }  // namespace
@@ -85,7 +92,7 @@ extern "C" size_t wal_body_workspace_bytes(const wal_matrix* mats, int n_mats, i
   if (!mats || n_mats <= 0 || M < 1) return 0;
   for (int i = 0; i < n_mats; ++i)
     if (!wal_workspace_bytes(&mats[i], M)) return 0;
-  return 512;  // status header only: the batch-1 kernels keep every intermediate on chip
+  return body_ws_total(n_mats, M);
 }
 
 extern "C" int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n_mats, const int32_t* stage_of,
@@ -113,6 +120,10 @@ extern "C" int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n
       }
       *plan = p;
     }
+    // the previous graph may still be running on `stream` and reading the
+    // launch tables in the workspace
+    cudaError_t se = cudaStreamSynchronize((cudaStream_t)stream);
+    if (se != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("stream synchronize: ") + cudaGetErrorString(se));
     release(p);
     p->mats.assign(mats, mats + n_mats);
     p->stages.assign(stage_of, stage_of + n_mats);
@@ -122,37 +133,50 @@ extern "C" int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n
     p->ws = ws;
     p->ws_bytes = ws_bytes;
 
-    cudaError_t e = cudaStreamBeginCapture(p->capture_stream, cudaStreamCaptureModeThreadLocal);
-    if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("begin capture: ") + cudaGetErrorString(e));
-    int st = WAL_OK;
-    const std::vector<LaunchGroup> groups = group_launches(mats, n_mats, stage_of, M);
-    for (size_t gi = 0; gi < groups.size() && st == WAL_OK; ++gi) {
-      const LaunchGroup& lg = groups[gi];
-      StreamParams prm = {};
-      prm.K = mats[lg.first].K;
-      prm.status = reinterpret_cast<int32_t*>(align_up((uintptr_t)ws, 256));
-      int n_items = 0;
+    // launch tables: groups and items, uploaded into the workspace
+    const std::vector<LaunchGroup> lgs = group_launches(mats, n_mats, stage_of, M);
+    std::vector<GroupDesc> groups(lgs.size());
+    std::vector<StreamItem> items;
+    items.reserve((size_t)n_mats * M);
+    for (size_t gi = 0; gi < lgs.size(); ++gi) {
+      const LaunchGroup& lg = lgs[gi];
+      const int item0 = (int)items.size();
       for (int i = lg.first; i < lg.first + lg.count; ++i)
         for (int mi = 0; mi < M; ++mi)
-          prm.items[n_items++] = make_item(&mats[i], xs[i] + (size_t)mi * mats[i].K, ys[i] + (size_t)mi * mats[i].N);
-      prm.n_items = n_items;
-      // warm L2 with the weights of the next launch
-      if (gi + 1 < groups.size()) {
-        const LaunchGroup& nx = groups[gi + 1];
-        int n_pf = 0;
-        for (int i = nx.first; i < nx.first + nx.count; ++i) {
-          size_t sz[6];
-          sizes_of(mats[i].N, mats[i].K, mats[i].k, mats[i].r, sz);
-          n_pf = add_prefetch(prm.pf, n_pf, mats[i].codes, sz[0]);
-          n_pf = add_prefetch(prm.pf, n_pf, mats[i].sites, sz[1]);
-          n_pf = add_prefetch(prm.pf, n_pf, mats[i].scales, sz[2]);
-        }
-        prm.n_pf = n_pf;
-      }
-      StreamLaunch L;
-      st = plan_stream(prm.items, n_items, prm.K, &L);
-      if (st == WAL_OK) st = launch_stream(prm, L, p->capture_stream, gi > 0);
+          items.push_back(make_item(&mats[i], xs[i] + (size_t)mi * mats[i].K, ys[i] + (size_t)mi * mats[i].N));
+      int st = plan_group(items.data() + item0, (int)items.size() - item0, mats[lg.first].K, &groups[gi]);
+      if (st) return st;
+      groups[gi].item0 = item0;
+      // stages renumbered 0, 1, 2, ... (only changes matter to the launch)
+      groups[gi].stage = gi == 0 ? 0 : groups[gi - 1].stage + (stage_of[lg.first] != stage_of[lgs[gi - 1].first]);
     }
+    StreamLaunch L;
+    int st = plan_launch(groups.data(), (int)groups.size(), true, &L);
+    if (st) return st;
+    if (L.grid > kMaxCtas) return fail(WAL_ERR_UNSUPPORTED, "more than 1024 SMs");
+    const int ng = (int)groups.size();
+    std::vector<TileRec> sched((size_t)L.grid * ng);
+    for (int b = 0; b < L.grid; ++b) build_schedule(groups.data(), ng, items.data(), b, sched.data() + (size_t)b * ng);
+    char* base = reinterpret_cast<char*>(align_up((uintptr_t)ws, 256));
+    cudaError_t e = cudaMemcpy(base + items_offset(), items.data(), items.size() * sizeof(StreamItem),
+                               cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(base + sched_offset(n_mats, M), sched.data(), sched.size() * sizeof(TileRec),
+                     cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("launch-table upload: ") + cudaGetErrorString(e));
+    StreamParams prm = {};
+    prm.t_sched = reinterpret_cast<const TileRec*>(base + sched_offset(n_mats, M));
+    prm.t_items = reinterpret_cast<const StreamItem*>(base + items_offset());
+    prm.n_groups = ng;
+    prm.barrier = reinterpret_cast<unsigned int*>(base + kBarrierOffset);
+    prm.status = reinterpret_cast<int32_t*>(base);
+
+    e = cudaStreamBeginCapture(p->capture_stream, cudaStreamCaptureModeThreadLocal);
+    if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("begin capture: ") + cudaGetErrorString(e));
+    // status word and barrier counter start at zero on every replay
+    e = cudaMemsetAsync(base, 0, 256, p->capture_stream);
+    if (e != cudaSuccess) st = fail(WAL_ERR_CUDA, std::string("header clear: ") + cudaGetErrorString(e));
+    if (st == WAL_OK) st = launch_body(prm, L, p->capture_stream);
     cudaGraph_t g = nullptr;
     e = cudaStreamEndCapture(p->capture_stream, &g);
     if (st != WAL_OK) {

@@ -143,21 +143,20 @@ StreamItem make_item(const wal_matrix* m, const uint16_t* x, float* y) {
   return it;
 }
 
-// Products of one matrix for activation rows [m0, m0 + count) in one launch.
+// Products of one matrix for activation rows [m0, m0 + count) in one launch
+// (one group: every product shares K).
 int launch_rows(const wal_matrix* m, const uint16_t* X, int ldx, float* Y, int ldy, int m0, int count,
-                cudaStream_t stream, bool pdl, const PrefetchRange* pf, int n_pf, int32_t* status) {
+                cudaStream_t stream, int32_t* status) {
   StreamParams prm = {};
   prm.status = status;
-  prm.n_items = count;
-  prm.K = m->K;
   for (int i = 0; i < count; ++i)
     prm.items[i] = make_item(m, X + (size_t)(m0 + i) * ldx, Y + (size_t)(m0 + i) * ldy);
-  prm.n_pf = n_pf;
-  for (int j = 0; j < n_pf; ++j) prm.pf[j] = pf[j];
-  StreamLaunch L;
-  int st = plan_stream(prm.items, count, m->K, &L);
+  int st = plan_group(prm.items, count, m->K, &prm.group);
   if (st) return st;
-  return launch_stream(prm, L, stream, pdl);
+  StreamLaunch L;
+  st = plan_launch(&prm.group, 1, false, &L);
+  if (st) return st;
+  return launch_stream(prm, L, stream);
 }
 
 size_t product_ws_bytes(const wal_matrix* m, int M) {
@@ -197,8 +196,7 @@ extern "C" int wal_gemv(const wal_matrix* m, const uint16_t* x, float* y, void* 
   if (st) return st;
   st = ws_check(ws, ws_bytes, product_ws_bytes(m, 1));
   if (st) return st;
-  return launch_rows(m, x, m->K, y, m->N, 0, 1, (cudaStream_t)stream, false, nullptr, 0,
-                     reinterpret_cast<int32_t*>(ws_base(ws)));
+  return launch_rows(m, x, m->K, y, m->N, 0, 1, (cudaStream_t)stream, reinterpret_cast<int32_t*>(ws_base(ws)));
 }
 
 extern "C" int wal_gemm_small_m(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, int ldy,
@@ -210,7 +208,7 @@ extern "C" int wal_gemm_small_m(const wal_matrix* m, const uint16_t* X, int M, i
   // more than 16 activation rows: the product is a dense contraction (tensor cores)
   if (M > kMaxItems) return launch_tc(m, X, M, ldx, Y, ldy, ws_base(ws), (cudaStream_t)stream);
   for (int m0 = 0; m0 < M; m0 += kMaxItems) {
-    st = launch_rows(m, X, ldx, Y, ldy, m0, std::min(kMaxItems, M - m0), (cudaStream_t)stream, false, nullptr, 0,
+    st = launch_rows(m, X, ldx, Y, ldy, m0, std::min(kMaxItems, M - m0), (cudaStream_t)stream,
                      reinterpret_cast<int32_t*>(ws_base(ws)));
     if (st) return st;
   }

@@ -2,45 +2,51 @@
 //   y = (alpha*T + beta*R) x + sum_r s_r U_r (V_r^T x)
 // (WAL-Ternary-8B model card, "Representation").
 //
-// One launch processes a work list of up to kMaxItems products that share K
-// (for example the q, k and v matrices of one dependency stage).  One CTA owns
-// one tile = RB consecutive output rows of one product and every K-slice of
-// them, so nothing leaves the CTA before y is written.
+// One launch runs a list of groups.  A group is up to kMaxItems products that
+// share K; one CTA owns one tile of a group = RB consecutive output rows of
+// one product and every K-slice of them, so nothing leaves the CTA before y
+// is written.  A single product call is one group.  A body pass is one
+// persistent, cooperative launch over all its groups, one CTA per SM: groups
+// of one dependency stage follow each other directly, and between stages the
+// CTAs meet at a grid barrier (stage s + 1 may read what stage s wrote).
 //
 // A lane owns one 128-group of a row (8 code words), a warp a K-slice of 4096
-// columns; the CTA has S slices x P phases warps.
-//  1. x first: every thread requests its chunks of x (after the dependent-
-//     launch wait, since x may be the previous stage's output).  Then lane 0
-//     of each warp starts the warp's TMA ring: per row of the warp, one bulk
-//     copy of the slice's code bytes (32 lanes x 32 B), one of its residual-
-//     site bytes and one of its {alpha, beta} words, completing on an
-//     mbarrier per ring stage (two rows).  The WALB2 bit planes (V) and bit
-//     words (U) of the tile follow by cp.async.
-//  2. The CTA builds the fixed-point image of x: per group g with largest
-//     exponent e_g, X_j = round(x_j * 2^(21 - e_g)), an integer below 2^22 in
-//     magnitude (exact when x_j is within 2^-14 of the group maximum, round-
-//     to-nearest-even below that), as three byte limbs per column, with the
-//     group sum of X, the group weight 2^(e_g - 21) and a +-X table indexed
-//     by the raw residual-site byte.  The table is interleaved by group so
-//     that the lanes of a warp (one group each) never share a bank when they
-//     look up their sites; it is filled through a padded transpose.
-//  3. Each lane pulls its 96 limb words into registers.  The trit decode masks
-//     each code word once per slot (word & (0x03030303 << 2s) leaves 4^s times
-//     the code t + 1 of trit 4b + s in byte b); three dp4a per slot against
-//     the lo / mid / hi limbs accumulate per slot, and exact shifts fold the
-//     slots, giving sum_j (t_j + 1) X_j; minus sum_j X_j that is T.x of the
-//     group in int32.  The residual sites add +-X from the table (exact).
-//     alpha and beta are applied in FP32 and the group weight once.  The
-//     WALB2 phase-1 products V_r^T x go through the same path: a row of V is
-//     a ternary row without zeros, its bits spread into 2-bit codes.
-//  4. Each lane leaves its group's partial in shared memory; after the rows
-//     one thread per output row sums the slices and lanes in a fixed order,
-//     and the WALB2 phase-2 term sum_r U[n, r] z_r joins in the single store.
-// Results are bitwise reproducible: no atomics, fixed reduction orders.
-// Every mbarrier wait is bounded; a wait that gives up records
-// WAL_ERR_TIMEOUT in the status word and the warp skips the rest of its rows.
+// columns; a group uses S slices x P phases warps.
+//  - Weights stream through a per-warp TMA ring that runs ahead across group
+//    and stage boundaries (the weights do not depend on x): lane 0 of each
+//    warp keeps `stages` chunks of two rows in flight, one bulk copy each for
+//    a row's code bytes (32 lanes x 32 B), residual-site bytes and
+//    {alpha, beta} words, completing on an mbarrier per ring slot.  While a
+//    CTA waits at the grid barrier its ring already fills with the next
+//    stage's rows; an L2 prefetch of its next tile, issued once its rows of
+//    the current group are consumed, keeps HBM busy through the combine, the
+//    barrier and the next prep.
+//  - Per group the CTA builds the fixed-point image of x: per 128-group g
+//    with largest exponent e_g, X_j = round(x_j * 2^(21 - e_g)), an integer
+//    below 2^22 in magnitude (exact when x_j is within 2^-14 of the group
+//    maximum, round-to-nearest-even below that), as three byte limbs per
+//    column, with the group sum of X, the group weight 2^(e_g - 21) and a
+//    table of X (or X then -X) indexed by the residual-site byte, group-major
+//    with an odd stride so the lanes of a warp (one group each) spread over
+//    the banks.  One pass over x and one CTA barrier.
+//  - Each lane pulls its 96 limb words into registers.  The trit decode
+//    masks each code word once per slot (word & (0x03030303 << 2s) leaves
+//    4^s times the code t + 1 of trit 4b + s in byte b); three dp4a per slot
+//    against the lo / mid / hi limbs accumulate per slot, and exact shifts
+//    fold the slots, giving sum_j (t_j + 1) X_j; minus sum_j X_j that is T.x
+//    of the group in int32.  The residual sites add +-X from the table
+//    (exact).  alpha and beta are applied in FP32 and the group weight once.
+//    The WALB2 phase-1 products V_r^T x go through the same path: a row of
+//    V is a ternary row without zeros, its bits spread into 2-bit codes.
+//  - Each lane leaves its group's partial in shared memory; after the rows
+//    one thread per output row sums the slices and lanes in a fixed order,
+//    and the WALB2 phase-2 term sum_r U[n, r] z_r joins in the single store.
+// Results are bitwise reproducible: no atomics in the arithmetic, fixed
+// reduction orders.  Every wait (mbarrier, grid barrier) is bounded; one that
+// gives up records WAL_ERR_TIMEOUT in the status word and the waiter moves on.
 #include "wal_internal.h"
 #include "wal_device.cuh"
+#include "wal_ptx.cuh"
 #include "wal_stream.h"
 
 #include <algorithm>
@@ -49,26 +55,32 @@
 namespace wal {
 
 using namespace dev;
+using ptx::mbar_init;
+using ptx::mbar_arrive_expect_tx;
+using ptx::mbar_wait;
+using ptx::bulk_g2s;
 
-constexpr int kRowsPerStage = 2;
+constexpr int kRowsPerStage = 3;  // rows per ring chunk
 constexpr int kMaxThreads = 384;
+constexpr int kMaxWarps = kMaxThreads / 32;
 constexpr int kMaxXChunks = 8;            // 8-column chunks of x per thread
 constexpr uint32_t kMagic = 0x4B400000u;  // 1.5 * 2^23: adding it rounds |v| < 2^22 to an integer
-constexpr uint32_t kSpinLimit = 1u << 22; // try_wait polls before a wait gives up
 constexpr uint32_t kLimbStride = 100;     // words per group in the limb image (96 + 4 pad)
-// one row of one warp in the ring: codes 32 x 32 B, sites 32 x 8 B (+16 B
-// alignment slack), scales 32 x 4 B (+16 B slack)
-constexpr uint32_t kSlotCodes = 0, kSlotSites = 1024, kSlotScales = 1024 + 272, kSlotBytes = 1024 + 272 + 144;
+constexpr uint32_t kPartStride = 33;      // floats per row of per-lane partials (32 + 1 pad: the combine reads a row per thread)
+constexpr uint32_t kBarrierSpin = 1u << 22;  // polls of the grid-barrier counter before giving up
+// One ring chunk of one warp: three rows of codes (32 lanes x 32 B each), then
+// their site bytes (32 x 8 B each + 16 B alignment slack), then their
+// {alpha, beta} words (32 x 4 B each + 16 B slack).  With a single K-slice
+// (K <= 4096) the three rows are contiguous in every buffer and arrive as one
+// copy per buffer, packed at the buffers' own row pitch; otherwise each row is
+// copied on its own at the fixed pitches below.
+constexpr uint32_t kCodePitch = 1024, kSitePitch = 272, kScalePitch = 144;
+constexpr uint32_t kChunkSites = kRowsPerStage * kCodePitch;
+constexpr uint32_t kChunkScales = kChunkSites + kRowsPerStage * kSitePitch;
+constexpr uint32_t kChunkBytes = kChunkScales + kRowsPerStage * kScalePitch;
 
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-// ---- raw shared-memory access (32-bit shared-window addresses) -------------
-__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 __device__ __forceinline__ void cp_async4_zfill(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
@@ -76,16 +88,6 @@ __device__ __forceinline__ void cp_async4_zfill(uint32_t dst, const void* src, u
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
 __device__ __forceinline__ uint32_t lds16(uint32_t a) {
@@ -98,36 +100,19 @@ __device__ __forceinline__ int32_t ldsi(uint32_t a) {
   asm volatile("ld.shared.s32 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
+// x may have been written by an earlier stage of the same launch: read it at
+// L2 (coherent), never through the non-coherent or L1 path.
+__device__ __forceinline__ uint4 ld_cg128(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_acquire(const unsigned int* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 __device__ __forceinline__ uint32_t byte_of(uint32_t w, int b) { return __byte_perm(w, 0u, 0x4440u | (uint32_t)b); }
-
-// ---- mbarrier + bulk copies (one CTA is its own cluster) -------------------
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(done)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-// Bounded wait: false (and the status word set) if the phase never completes.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* status) {
-  for (uint32_t it = 0; it < kSpinLimit; ++it)
-    if (mbar_try_wait(bar, parity)) return true;
-  if (status) atomicExch(status, (int32_t)WAL_ERR_TIMEOUT);
-  return false;
-}
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
-}
 
 // 16 bits -> the even bit positions of a 32-bit word.
 __device__ __forceinline__ uint32_t spread16(uint32_t x) {
@@ -160,389 +145,500 @@ __device__ __forceinline__ int32_t group_dot(const uint32_t (&wv)[8], const uint
   return (int32_t)(((uint32_t)t2 << 16) + (t1 << 8) + t0);
 }
 
-struct SmemPlan {
-  uint32_t table, limbs, xgsum, gsc, partz, part, vstage, ubuf, scratch, ring, mbar, total;
+// ---------------------------------------------------------------------------
+// shared memory: [ring | mbarriers | producer states] then the per-group area
+// ---------------------------------------------------------------------------
+// Site table: per group, the X of its 128 columns (and, in the signed
+// table, their negations after them), group-major with an odd stride so
+// that groups land on different banks.
+__host__ __device__ inline uint32_t table_stride(bool signed_table) { return signed_table ? 257u : 129u; }
+
+__host__ __device__ inline uint32_t ring_bytes(int warps, int stages) {
+  return (uint32_t)warps * stages * kChunkBytes;
+}
+struct ProdState;  // defined below
+__host__ __device__ inline uint32_t area_offset(int warps, int stages);
+
+struct AreaPlan {
+  uint32_t table, limbs, part, xgsum, gsc, partz, ubuf, vstage, total;
 };
-
-// Groups rounded up to a multiple of 32: the +-X table is interleaved as
-// [entry][group], so lane l of a warp (group 32 s + l) always reads bank l.
-__host__ __device__ inline uint32_t group_stride(int K) { return (uint32_t)((K / kGroup + 31) / 32 * 32); }
-
-// Shared-memory carve-up of one CTA.
-__host__ __device__ inline SmemPlan smem_plan(int K, int threads, int S, int RB, int rmax, bool signed_table,
-                                              int stages, bool stage_v) {
-  SmemPlan p;
+// Carve-up of the per-group area (offsets relative to the area base).  The
+// limb image is dead once every warp holds its limbs in registers; the
+// per-lane partials, written only after that, reuse its space.
+__host__ __device__ inline AreaPlan area_plan(int K, int S, int RB, bool signed_table) {
+  AreaPlan p;
   uint32_t off = 0;
   auto take = [&](uint32_t bytes) { uint32_t o = off; off = (off + bytes + 15u) & ~15u; return o; };
   const uint32_t G = (uint32_t)K / kGroup;
-  p.table = take(group_stride(K) * (signed_table ? 256u : 128u) * 4u);
-  p.limbs = take(G * kLimbStride * 4u);
+  p.table = take(G * table_stride(signed_table) * 4u);
+  const uint32_t limbs = G * kLimbStride * 4u, part = (uint32_t)S * RB * kPartStride * 4u;
+  p.limbs = p.part = take(part > limbs ? part : limbs);
   p.xgsum = take(G * 4u);
   p.gsc = take(G * 4u);
   p.partz = take((uint32_t)S * WAL_MAX_RANK * 4u);
-  p.part = take((uint32_t)S * RB * 32u * 4u);  // per-lane partials [slice][row][lane]
-  p.vstage = take(stage_v ? (uint32_t)rmax * (uint32_t)(K / 8) : 0u);
-  p.ubuf = take((uint32_t)RB * 4u);             // U bit words of the tile's rows
-  p.scratch = take(32u * 129u * 4u);            // X of 32 groups, rows padded to 129 words
-  p.ring = take((uint32_t)(threads / 32) * stages * kRowsPerStage * kSlotBytes);
-  p.mbar = take((uint32_t)(threads / 32) * stages * 8u);
+  p.ubuf = take((uint32_t)RB * 4u);
+  // V bit planes of the first P ranks (each of the P phases of a slice takes one): P * K / 8 bytes
+  p.vstage = take((uint32_t)(kMaxWarps / S) * (uint32_t)K / 8u);
   p.total = off;
   return p;
 }
 
-// One warp's view of its rows: row i of the warp is output row n0 + p + P i.
+// Rows of one warp in one group: a contiguous block, row i of the warp is
+// output row nb + i of one product (tile row r0 + i), columns of K-slice s.
 struct WarpRing {
-  uint32_t ring;   // warp's ring base (shared window)
-  uint32_t mbar;   // warp's mbarriers
-  int stages;
+  const uint32_t* codes;
+  const uint8_t* sites;
+  const uint16_t* scales;
   int nmine;
-  int s, p, P, n0, G, K, k;
-  const StreamItem* it;
-  __device__ __forceinline__ uint32_t slot(int stage, int u) const {
-    return ring + ((uint32_t)stage * kRowsPerStage + (uint32_t)u) * kSlotBytes;
-  }
-  __device__ __forceinline__ uint32_t bar(int stage) const { return mbar + (uint32_t)stage * 8u; }
-  // groups of the warp's slice, and the group index of the slice's first group in row i
+  int s, nb, r0, G, K, k;
+  __device__ __forceinline__ bool one_slice() const { return G <= 32; }
   __device__ __forceinline__ int ngroups() const { return min(32, G - 32 * s); }
-  __device__ __forceinline__ size_t gbase(int i) const { return (size_t)(n0 + p + P * i) * G + 32 * s; }
 };
+
+// What warp `warp` does for tile record t of product `it` (nmine = 0: nothing).
+// `it` is read only when the record has rows.  The P warps of a slice take
+// contiguous blocks of ceil(rows / P) rows.
+__device__ __forceinline__ void warp_work(const TileRec& t, const StreamItem* it, int warp, WarpRing& W) {
+  W.codes = nullptr; W.sites = nullptr; W.scales = nullptr;
+  W.nmine = 0;
+  W.s = W.r0 = 0;
+  W.nb = t.n0;
+  W.G = t.G; W.K = (int)t.G * kGroup; W.k = 0;
+  if (t.rows == 0 || warp >= (int)t.S * t.P) return;
+  W.codes = it->codes; W.sites = it->sites; W.scales = it->scales; W.k = it->k;
+  W.s = warp % t.S;
+  const int p = warp / t.S, m = ((int)t.rows + t.P - 1) / t.P;
+  W.r0 = p * m;
+  W.nb = t.n0 + W.r0;
+  W.nmine = max(0, min(m, (int)t.rows - W.r0));
+}
+
+// Host and device: the tile record of CTA `cta` in group g.
+__host__ __device__ inline TileRec tile_record(const GroupDesc& g, const StreamItem* items, int cta) {
+  TileRec t = {};
+  t.G = (uint8_t)(g.K / kGroup); t.S = (uint8_t)g.S; t.P = (uint8_t)g.P;
+  t.signed_table = (uint8_t)g.signed_table;
+  t.RB = (uint16_t)g.RB;
+  t.stage = (uint16_t)g.stage;
+  if (cta >= g.tiles) return t;
+  int i = 0;
+  while (i + 1 < g.n_items && cta >= items[i + 1].tile_begin) ++i;
+  const int n0 = (cta - items[i].tile_begin) * g.RB;
+  const int rows = items[i].N - n0 < g.RB ? items[i].N - n0 : g.RB;
+  t.item = (uint16_t)(g.item0 + i);
+  t.n0 = n0;
+  t.rows = (uint16_t)rows;
+  return t;
+}
 
 __device__ __forceinline__ uint32_t site_bytes(int k) { return (uint32_t)k; }
 __device__ __forceinline__ uint32_t scale_bytes(int k) { return k > 0 ? 4u : 2u; }
 
-// Lane 0: queue the rows of chunk `chunk` (two rows) into ring stage `stage`.
-// Site and scale ranges are widened to 16-byte boundaries (every buffer is
-// zero-padded to a multiple of 16 bytes, so the widened range stays inside).
-__device__ __forceinline__ void issue_chunk(const WarpRing& W, int stage, int chunk) {
-  const int ng = W.ngroups();
+// Queue the rows of chunk `chunk` of W into ring slot `sl` with mbarrier
+// `bar`.  Site and scale ranges are widened to 16-byte boundaries (every
+// buffer is zero-padded to a multiple of 16 bytes, so the widened range stays
+// inside).
+__device__ __forceinline__ void issue_chunk(const WarpRing& W, uint32_t sl, uint32_t bar, int chunk) {
+  const int i0 = chunk * kRowsPerStage;
+  const int un = min(kRowsPerStage, W.nmine - i0);
+  if (un <= 0) return;
   const uint32_t kb = site_bytes(W.k), sb = scale_bytes(W.k);
-  const unsigned char* src[kRowsPerStage][3];
-  uint32_t len[kRowsPerStage][3];
-  uint32_t bytes = 0;
-#pragma unroll
-  for (int u = 0; u < kRowsPerStage; ++u) {
-    const int i = chunk * kRowsPerStage + u;
-    len[u][0] = len[u][1] = len[u][2] = 0u;
-    src[u][0] = src[u][1] = src[u][2] = nullptr;
-    if (i < W.nmine) {
-      const size_t n = (size_t)(W.n0 + W.p + W.P * i);
-      const size_t gb = W.gbase(i);
-      src[u][0] = reinterpret_cast<const unsigned char*>(W.it->codes) + n * (size_t)(W.K / 4) + (size_t)W.s * 1024;
-      len[u][0] = (uint32_t)ng * 32u;
-      if (W.k > 0) {
-        const size_t a = (gb * kb) & ~(size_t)15, e = ((gb + ng) * kb + 15) & ~(size_t)15;
-        src[u][1] = W.it->sites + a;
-        len[u][1] = (uint32_t)(e - a);
-      }
-      const size_t a = (gb * sb) & ~(size_t)15, e = ((gb + ng) * sb + 15) & ~(size_t)15;
-      src[u][2] = reinterpret_cast<const unsigned char*>(W.it->scales) + a;
-      len[u][2] = (uint32_t)(e - a);
-      bytes += len[u][0] + len[u][1] + len[u][2];
-    }
+  const unsigned char* cbase = reinterpret_cast<const unsigned char*>(W.codes);
+  const unsigned char* abase = reinterpret_cast<const unsigned char*>(W.scales);
+  if (W.one_slice()) {
+    const size_t n = (size_t)(W.nb + i0), G = (size_t)W.G;
+    const uint32_t clen = (uint32_t)un * (uint32_t)(W.K / 4);
+    const size_t sa = (n * G * kb) & ~(size_t)15, se = ((n + un) * G * kb + 15) & ~(size_t)15;
+    const size_t aa = (n * G * sb) & ~(size_t)15, ae = ((n + un) * G * sb + 15) & ~(size_t)15;
+    mbar_arrive_expect_tx(bar, clen + (uint32_t)(se - sa) + (uint32_t)(ae - aa));
+    bulk_g2s(sl, cbase + n * (size_t)(W.K / 4), clen, bar);
+    if (se > sa) bulk_g2s(sl + kChunkSites, W.sites + sa, (uint32_t)(se - sa), bar);
+    bulk_g2s(sl + kChunkScales, abase + aa, (uint32_t)(ae - aa), bar);
+    return;
   }
-  if (bytes == 0) return;
-  const uint32_t bar = W.bar(stage);
+  // several K-slices: each row on its own (lengths first for the expected bytes)
+  const int ng = W.ngroups();
+  auto site_range = [&](size_t gb, size_t& a, size_t& e) {
+    a = (gb * kb) & ~(size_t)15;
+    e = ((gb + ng) * kb + 15) & ~(size_t)15;
+  };
+  auto scale_range = [&](size_t gb, size_t& a, size_t& e) {
+    a = (gb * sb) & ~(size_t)15;
+    e = ((gb + ng) * sb + 15) & ~(size_t)15;
+  };
+  uint32_t bytes = 0;
+  for (int u = 0; u < un; ++u) {
+    const size_t gb = (size_t)(W.nb + i0 + u) * W.G + 32 * W.s;
+    size_t a, e, a2, e2;
+    site_range(gb, a, e);
+    scale_range(gb, a2, e2);
+    bytes += (uint32_t)ng * 32u + (uint32_t)(e - a) + (uint32_t)(e2 - a2);
+  }
   mbar_arrive_expect_tx(bar, bytes);
-#pragma unroll
-  for (int u = 0; u < kRowsPerStage; ++u) {
-    if (len[u][0] == 0u) continue;
-    const uint32_t sl = W.slot(stage, u);
-    bulk_g2s(sl + kSlotCodes, src[u][0], len[u][0], bar);
-    if (len[u][1]) bulk_g2s(sl + kSlotSites, src[u][1], len[u][1], bar);
-    bulk_g2s(sl + kSlotScales, src[u][2], len[u][2], bar);
+  for (int u = 0; u < un; ++u) {
+    const size_t n = (size_t)(W.nb + i0 + u);
+    const size_t gb = n * W.G + 32 * W.s;
+    size_t a, e, a2, e2;
+    site_range(gb, a, e);
+    scale_range(gb, a2, e2);
+    bulk_g2s(sl + (uint32_t)u * kCodePitch, cbase + n * (size_t)(W.K / 4) + (size_t)W.s * 1024, (uint32_t)ng * 32u, bar);
+    if (e > a) bulk_g2s(sl + kChunkSites + (uint32_t)u * kSitePitch, W.sites + a, (uint32_t)(e - a), bar);
+    bulk_g2s(sl + kChunkScales + (uint32_t)u * kScalePitch, abase + a2, (uint32_t)(e2 - a2), bar);
   }
 }
 
-// tab = table base + 4 * group; entries of one group are gstride4 bytes apart
+// The producer side of a warp's ring (kept in shared memory, used by lane 0):
+// the next chunk to issue, which may lie in a later group.
+struct ProdState {
+  int j, c, nc;
+  uint32_t issued;    // chunks issued so far
+  uint32_t consumed;  // chunks consumed so far
+  WarpRing W;
+};
+__host__ __device__ inline uint32_t area_offset(int warps, int stages) {
+  const uint32_t o = ring_bytes(warps, stages) + (uint32_t)warps * stages * 8u +
+                     (uint32_t)warps * (uint32_t)((sizeof(ProdState) + 15) & ~(size_t)15);
+  return (o + 127u) & ~127u;
+}
+
+// Move the producer to the first group at or after ps.j with rows for this warp.
+__device__ __forceinline__ void prod_seek(ProdState& ps, const TileRec* sched, int n_groups, const StreamItem* items,
+                                          int warp) {
+  while (ps.j < n_groups) {
+    const TileRec t = sched[ps.j];
+    if (t.rows && warp < (int)t.S * t.P) {
+      warp_work(t, items + t.item, warp, ps.W);
+      ps.nc = (ps.W.nmine + kRowsPerStage - 1) / kRowsPerStage;
+      ps.c = 0;
+      if (ps.nc > 0) return;
+    }
+    ++ps.j;
+  }
+}
+
+// Issue the producer's next chunk into ring slot st (if any is left).
+__device__ __forceinline__ void prod_issue(ProdState& ps, uint32_t ring, uint32_t mbar, uint32_t st,
+                                           const TileRec* sched, int n_groups, const StreamItem* items, int warp) {
+  if (ps.j >= n_groups) return;
+  issue_chunk(ps.W, ring + st * kChunkBytes, mbar + st * 8u, ps.c);
+  ++ps.issued;
+  if (++ps.c == ps.nc) {
+    ++ps.j;
+    prod_seek(ps, sched, n_groups, items, warp);
+  }
+}
+
+// tab = shared address of this lane's group in the site table
 template <bool SIGNED_TABLE>
-__device__ __forceinline__ int32_t site_at(uint32_t tab, uint32_t gstride4, uint32_t byte) {
-  if (SIGNED_TABLE) return ldsi(tab + byte * gstride4);
-  const int32_t v = ldsi(tab + (byte & 0x7Fu) * gstride4);
+__device__ __forceinline__ int32_t site_at(uint32_t tab, uint32_t byte) {
+  if (SIGNED_TABLE) return ldsi(tab + byte * 4u);
+  const int32_t v = ldsi(tab + (byte & 0x7Fu) * 4u);
   return (byte & 0x80u) ? -v : v;
 }
 
-// One row's contribution of this lane's group, read from the ring slot:
-// 2^(e_g - 21) * (alpha * T.X + beta * R.X).  `hsw` swaps the two 16-byte
+// One row's contribution of this lane's group: 2^(e_g - 21) * (alpha * T.X +
+// beta * R.X).  crow, srow, arow: shared addresses of the row's codes, site
+// bytes and scale words for lane 0 of the warp.  `hsw` swaps the two 16-byte
 // halves of the lane's code chunk (matching the limb registers), so that the
 // 32-byte-strided reads of a warp never share a bank.
 template <int KS, bool SIGNED_TABLE>
-__device__ __forceinline__ float row_value(uint32_t sl, uint32_t site_off, uint32_t scale_off, int lane,
-                                           uint32_t hsw, const uint32_t (&lb)[8][kLimbWords], int32_t xs,
-                                           float gsc, uint32_t tab, uint32_t gs4) {
-  const uint32_t cd = sl + kSlotCodes + (uint32_t)lane * 32u;
+__device__ __forceinline__ float row_value(uint32_t crow, uint32_t srow, uint32_t arow, int lane, uint32_t hsw,
+                                           const uint32_t (&lb)[8][kLimbWords], int32_t xs, float gsc,
+                                           uint32_t tab) {
+  const uint32_t cd = crow + (uint32_t)lane * 32u;
   const uint4 c0 = lds128(cd + hsw), c1 = lds128(cd + (hsw ^ 16u));
   const uint32_t wv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
   const int32_t tdot = group_dot(wv, lb) - xs;
   int32_t q = 0;
   if (KS == 8) {
-    const uint2 sw = lds64(sl + kSlotSites + site_off + (uint32_t)lane * 8u);
-    q = site_at<SIGNED_TABLE>(tab, gs4, byte_of(sw.x, 0)) + site_at<SIGNED_TABLE>(tab, gs4, byte_of(sw.x, 1)) +
-        site_at<SIGNED_TABLE>(tab, gs4, byte_of(sw.x, 2));
-    q += site_at<SIGNED_TABLE>(tab, gs4, byte_of(sw.x, 3)) + site_at<SIGNED_TABLE>(tab, gs4, byte_of(sw.y, 0)) +
-         site_at<SIGNED_TABLE>(tab, gs4, byte_of(sw.y, 1));
-    q += site_at<SIGNED_TABLE>(tab, gs4, byte_of(sw.y, 2)) + site_at<SIGNED_TABLE>(tab, gs4, byte_of(sw.y, 3));
+    const uint2 sw = ptx::lds64(srow + (uint32_t)lane * 8u);
+    q = site_at<SIGNED_TABLE>(tab, byte_of(sw.x, 0)) + site_at<SIGNED_TABLE>(tab, byte_of(sw.x, 1)) +
+        site_at<SIGNED_TABLE>(tab, byte_of(sw.x, 2));
+    q += site_at<SIGNED_TABLE>(tab, byte_of(sw.x, 3)) + site_at<SIGNED_TABLE>(tab, byte_of(sw.y, 0)) +
+         site_at<SIGNED_TABLE>(tab, byte_of(sw.y, 1));
+    q += site_at<SIGNED_TABLE>(tab, byte_of(sw.y, 2)) + site_at<SIGNED_TABLE>(tab, byte_of(sw.y, 3));
   } else if (KS == 4) {
-    const uint32_t sw = lds32(sl + kSlotSites + site_off + (uint32_t)lane * 4u);
-    q = site_at<SIGNED_TABLE>(tab, gs4, byte_of(sw, 0)) + site_at<SIGNED_TABLE>(tab, gs4, byte_of(sw, 1)) +
-        site_at<SIGNED_TABLE>(tab, gs4, byte_of(sw, 2)) + site_at<SIGNED_TABLE>(tab, gs4, byte_of(sw, 3));
+    const uint32_t sw = ptx::lds32(srow + (uint32_t)lane * 4u);
+    q = site_at<SIGNED_TABLE>(tab, byte_of(sw, 0)) + site_at<SIGNED_TABLE>(tab, byte_of(sw, 1)) +
+        site_at<SIGNED_TABLE>(tab, byte_of(sw, 2)) + site_at<SIGNED_TABLE>(tab, byte_of(sw, 3));
   } else if (KS == 2) {
-    const uint32_t sw = lds16(sl + kSlotSites + site_off + (uint32_t)lane * 2u);
-    q = site_at<SIGNED_TABLE>(tab, gs4, sw & 0xFFu) + site_at<SIGNED_TABLE>(tab, gs4, sw >> 8);
+    const uint32_t sw = lds16(srow + (uint32_t)lane * 2u);
+    q = site_at<SIGNED_TABLE>(tab, sw & 0xFFu) + site_at<SIGNED_TABLE>(tab, sw >> 8);
   }
   if (KS == 0) {
-    const float alpha = fp16_bits_to_float(lds16(sl + kSlotScales + scale_off + (uint32_t)lane * 2u));
+    const float alpha = fp16_bits_to_float(lds16(arow + (uint32_t)lane * 2u));
     return alpha * ((float)tdot * gsc);
   }
-  const uint32_t sc = lds32(sl + kSlotScales + scale_off + (uint32_t)lane * 4u);
+  const uint32_t sc = ptx::lds32(arow + (uint32_t)lane * 4u);
   const float alpha = fp16_bits_to_float(sc & 0xFFFFu), beta = fp16_bits_to_float(sc >> 16);
   return fmaf(alpha, (float)tdot, beta * (float)q) * gsc;
 }
 
+// Everything a warp needs to walk its ring.
+struct RingCtx {
+  uint32_t ring, mbar;  // this warp's ring slots and mbarriers (shared window)
+  int stages;
+  ProdState* ps;        // this warp's producer state
+  const TileRec* sched; // this CTA's schedule (shared memory)
+  const StreamItem* items;
+  int n_groups, warp;
+  bool items_global;    // items live in device memory (not kernel parameters)
+  int32_t* status;
+};
+
+// Consume this warp's rows of the current group (ring positions q, q+1, ...);
+// after each chunk lane 0 refills the slot with the producer's next chunk.
+// False when a wait gave up.
 template <int KS, bool SIGNED_TABLE>
-__device__ __forceinline__ void run_rows(const WarpRing& W, int RB, int lane, bool active, uint32_t hsw,
-                                         const uint32_t (&lb)[8][kLimbWords], int32_t xs, float gsc, uint32_t tab,
-                                         uint32_t gs4, float* part, int32_t* status) {
+__device__ __forceinline__ bool run_rows(const WarpRing& W, const RingCtx& R, uint32_t& st, uint32_t& parity, int RB,
+                                         int lane, bool active, uint32_t hsw, const uint32_t (&lb)[8][kLimbWords],
+                                         int32_t xs, float gsc, uint32_t tab, float* part) {
   const int nc = (W.nmine + kRowsPerStage - 1) / kRowsPerStage;
-  float* mine = part + ((size_t)W.s * RB + W.p) * 32 + lane;  // partial of row p + P i at mine[P i * 32]
+  float* mine = part + (W.s * RB + W.r0) * (int)kPartStride + lane;  // row i at mine[i * kPartStride]
   const uint32_t kb = site_bytes(KS), sb = scale_bytes(KS);
-  int stage = 0;
-  uint32_t parity = 0;
+  const bool one = W.one_slice();
+  const uint32_t G = (uint32_t)W.G;
+  // one slice: pitches of the packed rows; otherwise the fixed pitches
+  const uint32_t cp = one ? G * 32u : kCodePitch, sp = one ? G * kb : kSitePitch, ap = one ? G * sb : kScalePitch;
 #pragma unroll 1
   for (int j = 0; j < nc; ++j) {
-    if (!mbar_wait(W.bar(stage), parity, status)) return;
+    const uint32_t sl = R.ring + st * kChunkBytes;
+    if (!mbar_wait(R.mbar + st * 8u, parity, R.status)) return false;
+    // group index of the chunk's first row (this slice's first group)
+    const uint32_t gb0 = (uint32_t)(W.nb + j * kRowsPerStage) * G + 32u * (uint32_t)W.s;
 #pragma unroll
     for (int u = 0; u < kRowsPerStage; ++u) {
       const int i = j * kRowsPerStage + u;
       if (i < W.nmine) {  // uniform across the warp
-        const size_t gb = W.gbase(i);
-        const uint32_t site_off = (uint32_t)((gb * kb) & 15), scale_off = (uint32_t)((gb * sb) & 15);
-        mine[(size_t)W.P * i * 32] =
-            active ? row_value<KS, SIGNED_TABLE>(W.slot(stage, u), site_off, scale_off, lane, hsw, lb, xs, gsc, tab, gs4)
-                   : 0.f;
+        const uint32_t gb = one ? gb0 : gb0 + (uint32_t)u * G;
+        const uint32_t srow = sl + kChunkSites + (uint32_t)u * sp + ((gb * kb) & 15u);
+        const uint32_t arow = sl + kChunkScales + (uint32_t)u * ap + ((gb * sb) & 15u);
+        const float v =
+            row_value<KS, SIGNED_TABLE>(sl + (uint32_t)u * cp, srow, arow, lane, hsw, lb, xs, gsc, tab);
+        mine[i * (int)kPartStride] = active ? v : 0.f;
       }
     }
-    __syncwarp();  // every lane has consumed the stage before it is refilled
-    if (lane == 0) issue_chunk(W, stage, j + W.stages);
-    if (++stage == W.stages) {
-      stage = 0;
+    __syncwarp();  // every lane has consumed the slot before it is refilled
+    if (lane == 0) {
+      ++R.ps->consumed;
+      prod_issue(*R.ps, R.ring, R.mbar, st, R.sched, R.n_groups, R.items, R.warp);
+    }
+    if (++st == (uint32_t)R.stages) {
+      st = 0;
       parity ^= 1u;
     }
   }
+  return true;
 }
 
-template <bool SIGNED_TABLE, int STAGES>
-__global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_constant__ StreamParams prm) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ float s_z[WAL_MAX_RANK];
-  const int K = prm.K, S = prm.S, P = prm.P, RB = prm.RB;
-  const int G = K / kGroup;
-  const int threads = blockDim.x;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const SmemPlan sp = smem_plan(K, threads, S, RB, prm.rmax, SIGNED_TABLE, STAGES, prm.stage_v != 0);
-  int32_t* table = reinterpret_cast<int32_t*>(smem + sp.table);
-  uint32_t* limbs = reinterpret_cast<uint32_t*>(smem + sp.limbs);
-  int32_t* xgsum = reinterpret_cast<int32_t*>(smem + sp.xgsum);
-  float* gsc_s = reinterpret_cast<float*>(smem + sp.gsc);
-  float* partz = reinterpret_cast<float*>(smem + sp.partz);
-  float* part = reinterpret_cast<float*>(smem + sp.part);
-  uint32_t* vst = reinterpret_cast<uint32_t*>(smem + sp.vstage);
-  uint32_t* ubuf = reinterpret_cast<uint32_t*>(smem + sp.ubuf);
-  int32_t* scratch = reinterpret_cast<int32_t*>(smem + sp.scratch);
-  if (blockIdx.x == 0 && tid == 0 && prm.status) *prm.status = 0;  // this launch has seen no timeout
+// This thread's 8-column chunks of x (chunk tid + i * blockDim.x).
+__device__ __forceinline__ void load_x(const uint16_t* x, int K, uint4 (&xr)[kMaxXChunks]) {
+  const int n8 = K / 8;
+#pragma unroll
+  for (int i = 0; i < kMaxXChunks; ++i) {
+    const int c8 = (int)threadIdx.x + i * (int)blockDim.x;
+    xr[i] = c8 < n8 ? ld_cg128(reinterpret_cast<const uint4*>(x) + c8) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
 
-  // which product and which rows
-  int item = 0;
-  while (item + 1 < prm.n_items && (int)blockIdx.x >= prm.items[item + 1].tile_begin) ++item;
-  const StreamItem& it = prm.items[item];
-  const int n0 = ((int)blockIdx.x - it.tile_begin) * RB;
-  const int rows = min(RB, it.N - n0);
-  const int s = warp % S, p = warp / S;
-  const int col0 = s * kSliceCols + lane * kGroup;
-  const bool active = col0 < K;
-  const int g = active ? col0 >> 7 : 0;
-  const int nmine = p < rows ? (rows - p + P - 1) / P : 0;
-  const int r = it.r;
-  const int ks = it.k;
+template <bool SIGNED_TABLE>
+__device__ __forceinline__ void build_image(const uint4 (&xr)[kMaxXChunks], int K, unsigned char* area,
+                                            const AreaPlan& ap) {
+  const int threads = blockDim.x, tid = threadIdx.x, lane = tid & 31;
+  const uint32_t tstride = table_stride(SIGNED_TABLE);
+  int32_t* table = reinterpret_cast<int32_t*>(area + ap.table);
+  uint32_t* limbs = reinterpret_cast<uint32_t*>(area + ap.limbs);
+  int32_t* xgsum = reinterpret_cast<int32_t*>(area + ap.xgsum);
+  float* gsc_s = reinterpret_cast<float*>(area + ap.gsc);
+  const int n8 = K / 8;
+#pragma unroll
+  for (int i = 0; i < kMaxXChunks; ++i) {
+    // chunk c8 = tid + i * threads, as loaded; the 16 chunks of one group sit
+    // on 16 aligned lanes of one warp, so the test below is uniform across
+    // each half-warp and its shuffles stay complete
+    const int c8 = tid + i * threads;
+    if (c8 >= n8) continue;
+    const unsigned gmask = (lane & 16) ? 0xFFFF0000u : 0x0000FFFFu;
+    const int c = 8 * c8;
+    const uint4 raw = xr[i];
+    const uint32_t pr[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t m2 = 0u;  // largest |x| bit pattern, two bf16 lanes
+#pragma unroll
+    for (int q = 0; q < 4; ++q) m2 = __vmaxu2(m2, pr[q] & 0x7FFF7FFFu);
+    uint32_t mx = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+    for (int off = 8; off; off >>= 1) mx = max(mx, __shfl_xor_sync(gmask, mx, off));
+    uint32_t emax = mx >> 7;
+    emax = emax > 1u ? emax : 1u;  // exponent field of the group maximum (denormals as 1)
+    // X = round(x * 2^(148 - emax)); tiny groups are pre-scaled by 2^64 so the factor stays finite
+    const float pre = emax < 64u ? 18446744073709551616.0f : 1.0f;
+    const float scl = __uint_as_float((275u - emax - (emax < 64u ? 64u : 0u)) << 23);
+    int32_t X[8];
+    int32_t sum8 = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float xv = bf16_bits_to_float((pr[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
+      X[q] = (int32_t)(__float_as_uint(fmaf(xv * pre, scl, __uint_as_float(kMagic))) - kMagic);
+      sum8 += X[q];
+    }
+#pragma unroll
+    for (int off = 8; off; off >>= 1) sum8 += __shfl_xor_sync(gmask, sum8, off);
+    const int gg = c >> 7, pos = c & 127, wl = (c >> 4) & 7, h = (c >> 3) & 1;
+    // limb image [group][word-in-group][limb][slot] (+4 words of padding per
+    // group): byte b of (word wl, limb L, slot q) = limb L of column 16 wl + 4 b + q
+    uint16_t* img16 = reinterpret_cast<uint16_t*>(limbs + (size_t)gg * kLimbStride);
+#pragma unroll
+    for (int L2 = 0; L2 < 3; ++L2)
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        img16[((wl * 3 + L2) * 4 + q) * 2 + h] =
+            (uint16_t)__byte_perm((uint32_t)X[q], (uint32_t)X[4 + q], (uint32_t)(L2 | ((4 + L2) << 4)));
+    if ((c8 & 15) == 0) {
+      xgsum[gg] = sum8;
+      gsc_s[gg] = emax >= 22u ? __uint_as_float((emax - 21u) << 23) : __uint_as_float(1u << (emax + 1u));
+    }
+    // site table: entry e of group gg (e = site byte) at gg * stride + e
+    int32_t* trow = table + (size_t)gg * tstride + pos;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      trow[q] = X[q];
+      if (SIGNED_TABLE) trow[128 + q] = -X[q];
+    }
+  }
+  __syncthreads();
+}
 
+// Warm L2 with a tile (codes, sites, scales of its rows) and its x.
+__device__ __forceinline__ void prefetch_tile(const TileRec& t, const StreamItem& it) {
+  const int K = (int)t.G * kGroup;
+  const size_t G = t.G, n0 = (size_t)t.n0, n1 = (size_t)t.n0 + t.rows;
+  const size_t sb = it.k ? 4 : 2;
+  const size_t ranges[3][2] = {{n0 * (K / 4), n1 * (K / 4)}, {n0 * G * it.k, n1 * G * it.k}, {n0 * G * sb, n1 * G * sb}};
+  const unsigned char* base[3] = {reinterpret_cast<const unsigned char*>(it.codes), it.sites,
+                                  reinterpret_cast<const unsigned char*>(it.scales)};
+  for (int b = 0; b < 3; ++b) {
+    if (!base[b] || ranges[b][1] == ranges[b][0]) continue;
+    const size_t a = ranges[b][0] & ~(size_t)15, e = (ranges[b][1] + 15) & ~(size_t)15;
+    for (size_t o = a; o < e; o += 65536) prefetch_l2(base[b] + o, (uint32_t)min((size_t)65536, e - o));
+  }
+  prefetch_l2(it.x, (uint32_t)(K * 2));
+}
+
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
+// One group on this CTA (which owns the tile t of it).  Returns false (on
+// every thread) when some wait of the CTA gave up.
+template <bool SIGNED_TABLE>
+__device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int j, uint32_t& st, uint32_t& parity,
+                                         unsigned char* area, float* s_z) {
+  const int threads = blockDim.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int K = (int)t.G * kGroup, S = t.S, P = t.P, RB = t.RB, rows = t.rows, n0 = t.n0;
+  const StreamItem& it = R.items[t.item];
   WarpRing W;
-  W.ring = smem_addr(smem + sp.ring) + (uint32_t)warp * STAGES * kRowsPerStage * kSlotBytes;
-  W.mbar = smem_addr(smem + sp.mbar) + (uint32_t)warp * STAGES * 8u;
-  W.stages = STAGES;
-  W.nmine = nmine;
-  W.s = s; W.p = p; W.P = P; W.n0 = n0; W.G = G; W.K = K; W.k = ks;
-  W.it = &it;
-  if (lane == 0) {
-    for (int st = 0; st < STAGES; ++st) mbar_init(W.bar(st), 1u);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncwarp();
+  warp_work(t, &it, warp, W);
+  const int r = it.r, ks = it.k;
+  const bool worker = warp < S * P;
+  const AreaPlan ap = area_plan(K, S, RB, SIGNED_TABLE);
+  float* partz = reinterpret_cast<float*>(area + ap.partz);
+  float* part = reinterpret_cast<float*>(area + ap.part);
+  uint32_t* ubuf = reinterpret_cast<uint32_t*>(area + ap.ubuf);
 
-  // 1. x first (x may be the output of the previous stage: dependent-launch wait)
-  pdl_wait();
+  // x first (it may be the previous stage's output), then the U words of the
+  // tile's rows and the V bit planes of the first P ranks
   uint4 xr[kMaxXChunks];
-  {
-    const int n8 = K / 8;
-#pragma unroll
-    for (int i = 0; i < kMaxXChunks; ++i) {
-      const int c8 = tid + i * threads;
-      xr[i] = c8 < n8 ? __ldg(reinterpret_cast<const uint4*>(it.x) + c8) : make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-  // the warp's TMA ring: every stage queued at once
-  if (lane == 0)
-    for (int st = 0; st < STAGES; ++st) issue_chunk(W, st, st);
-  // WALB2 bit planes (V) and the tile's U words, by cp.async (one group)
-  if (prm.stage_v && r > 0) {
-    const int n16 = r * (K / 128);  // 16-byte pieces of the [r][K/32] bit planes
-    for (int i = tid; i < n16; i += threads) cp_async16_zfill(smem_addr(vst) + 16u * i, it.vbits + 4 * i, 16u);
-  }
-  if (r > 0)
+  load_x(it.x, K, xr);
+  const int rv = min(r, P);  // ranks staged in shared memory
+  if (r > 0) {
     for (int rl = tid; rl < rows; rl += threads)
-      cp_async4_zfill(smem_addr(ubuf + rl), it.ubits + (size_t)(n0 + rl) * ((r + 31) / 32), 4u);
+      cp_async4_zfill(ptx::smem_u32(ubuf + rl), it.ubits + (size_t)(n0 + rl) * ((r + 31) / 32), 4u);
+    for (int i = tid; i < rv * (K / 128); i += threads)
+      cp_async16(reinterpret_cast<void*>(area + ap.vstage + 16u * i), it.vbits + 4 * i);
+  }
   cp_async_commit();
-  pdl_trigger();
-  // warm L2 with the next stage's weights, spread over all CTAs
-  if (tid == 0 && prm.n_pf > 0) {
-    for (int j = 0; j < prm.n_pf; ++j) {
-      const unsigned long long bytes = prm.pf[j].bytes;
-      const unsigned long long chunk = ((bytes / gridDim.x) + 4095ull) & ~4095ull;
-      const unsigned long long b0 = chunk * blockIdx.x;
-      if (b0 >= bytes) continue;
-      const unsigned long long b1 = b0 + chunk < bytes ? b0 + chunk : bytes;
-      for (unsigned long long o = b0; o < b1; o += 65536ull) {
-        const unsigned long long len = (b1 - o) < 65536ull ? (b1 - o) : 65536ull;
-        prefetch_l2(static_cast<const char*>(prm.pf[j].ptr) + o, (uint32_t)len);
-      }
-    }
-  }
 
-  // 2. fixed-point image of x
-  const uint32_t Gp = group_stride(K);
-  // blocks of 32 groups: phase A converts x (16 threads per group), phase B
-  // transposes the block's X into the interleaved +-X table (lanes = groups)
-  for (int gb = 0; gb < G; gb += 32) {
-    const int nblk = min(32, G - gb);
-#pragma unroll
-    for (int i = 0; i < kMaxXChunks; ++i) {
-      // chunk c8 = tid + i * threads, as loaded above; the 16 threads of one
-      // group are 16 aligned lanes of one warp, so the test below is uniform
-      // across each half-warp and the half-warp shuffles stay complete
-      const int c8 = tid + i * threads;
-      if (c8 < gb * 16 || c8 >= (gb + nblk) * 16) continue;
-      const unsigned gmask = (lane & 16) ? 0xFFFF0000u : 0x0000FFFFu;
-      const int c = 8 * c8;
-      const uint4 raw = xr[i];
-      const uint32_t pr[4] = {raw.x, raw.y, raw.z, raw.w};
-      uint32_t m2 = 0u;  // largest |x| bit pattern, two bf16 lanes
-#pragma unroll
-      for (int q = 0; q < 4; ++q) m2 = __vmaxu2(m2, pr[q] & 0x7FFF7FFFu);
-      uint32_t mx = max(m2 & 0xFFFFu, m2 >> 16);
-#pragma unroll
-      for (int off = 8; off; off >>= 1) mx = max(mx, __shfl_xor_sync(gmask, mx, off));
-      uint32_t emax = mx >> 7;
-      emax = emax > 1u ? emax : 1u;  // exponent field of the group maximum (denormals as 1)
-      // X = round(x * 2^(148 - emax)); tiny groups are pre-scaled by 2^64 so the factor stays finite
-      const float pre = emax < 64u ? 18446744073709551616.0f : 1.0f;
-      const float scl = __uint_as_float((275u - emax - (emax < 64u ? 64u : 0u)) << 23);
-      int32_t X[8];
-      int32_t sum8 = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float xv = bf16_bits_to_float((pr[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
-        X[q] = (int32_t)(__float_as_uint(fmaf(xv * pre, scl, __uint_as_float(kMagic))) - kMagic);
-        sum8 += X[q];
-      }
-#pragma unroll
-      for (int off = 8; off; off >>= 1) sum8 += __shfl_xor_sync(gmask, sum8, off);
-      const int gg = c >> 7, pos = c & 127, wl = (c >> 4) & 7, h = (c >> 3) & 1;
-      // limb image [group][word-in-group][limb][slot] (+4 words of padding per
-      // group): byte b of (word wl, limb L, slot q) = limb L of column 16 wl + 4 b + q
-      uint16_t* img16 = reinterpret_cast<uint16_t*>(limbs + (size_t)gg * kLimbStride);
-#pragma unroll
-      for (int L2 = 0; L2 < 3; ++L2)
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          img16[((wl * 3 + L2) * 4 + q) * 2 + h] =
-              (uint16_t)__byte_perm((uint32_t)X[q], (uint32_t)X[4 + q], (uint32_t)(L2 | ((4 + L2) << 4)));
-      if ((c8 & 15) == 0) {
-        xgsum[gg] = sum8;
-        gsc_s[gg] = emax >= 22u ? __uint_as_float((emax - 21u) << 23) : __uint_as_float(1u << (emax + 1u));
-      }
-      int32_t* srow = scratch + (gg - gb) * 129 + pos;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) srow[q] = X[q];
-    }
-    __syncthreads();
-    // phase B: entry e of group gg at table[e * Gp + gg]; lane = group
-    if (lane < nblk)
-      for (int pos = warp; pos < 128; pos += threads / 32) {
-        const int32_t v = scratch[lane * 129 + pos];
-        table[(size_t)pos * Gp + gb + lane] = v;
-        if (SIGNED_TABLE) table[(size_t)(128 + pos) * Gp + gb + lane] = -v;
-      }
-    __syncthreads();
+  // the item records of the next groups into L1 (the producer reads them when it moves on)
+  if (R.items_global && tid < 4 && j + 1 + tid < R.n_groups) {
+    const TileRec tn = R.sched[j + 1 + tid];
+    if (tn.rows) prefetch_l1(R.items + tn.item);
   }
+  build_image<SIGNED_TABLE>(xr, K, area, ap);
 
-  // 3. the 96 limb words of this lane's group into registers; lanes with bit 2
+  // the 96 limb words of this lane's group into registers; lanes with bit 2
   // set swap the halves of their group (words 0-3 <-> 4-7), like their code reads
+  const int col0 = W.s * kSliceCols + lane * kGroup;
+  const bool active = worker && col0 < K;
+  const int g = active ? col0 >> 7 : 0;
   const uint32_t hsw = (lane & 4) ? 16u : 0u;
   uint32_t lb[8][kLimbWords];
   int32_t xs = 0;
   float gsc = 0.f;
   if (active) {
-    const uint4* img = reinterpret_cast<const uint4*>(limbs + (size_t)g * kLimbStride);
+    const uint32_t img = ptx::smem_u32(area + ap.limbs) + (uint32_t)g * kLimbStride * 4u;
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
       const int wsw = hsw ? (w ^ 4) : w;
 #pragma unroll
       for (int L2 = 0; L2 < 3; ++L2) {
-        const uint4 v = img[wsw * 3 + L2];
+        const uint4 v = lds128(img + (uint32_t)(wsw * 3 + L2) * 16u);
         lb[w][L2 * 4 + 0] = v.x; lb[w][L2 * 4 + 1] = v.y; lb[w][L2 * 4 + 2] = v.z; lb[w][L2 * 4 + 3] = v.w;
       }
     }
-    xs = xgsum[g];
-    gsc = gsc_s[g];
+    xs = reinterpret_cast<const int32_t*>(area + ap.xgsum)[g];
+    gsc = reinterpret_cast<const float*>(area + ap.gsc)[g];
   } else {
 #pragma unroll
     for (int w = 0; w < 8; ++w)
 #pragma unroll
-      for (int q = 0; q < kLimbWords; ++q) lb[w][q] = 0u;
+      for (int qq = 0; qq < kLimbWords; ++qq) lb[w][qq] = 0u;
   }
 
+  cp_async_wait<0>();
+  __syncthreads();  // staged U / V complete; the partials below overwrite the limb image
   // WALB2 phase 1: rows of V (no zeros: bit set -> code 0, clear -> code 2)
-  if (r > 0) {
-    cp_async_wait<0>();  // V planes and U words
-    __syncthreads();
-  }
-  for (int rho = p; rho < r; rho += P) {
-    float val = 0.f;
-    if (active) {
-      const uint32_t* vrow = (prm.stage_v ? vst : it.vbits) + (size_t)rho * (K / 32) + (size_t)g * 4;
-      const uint4 vb = *reinterpret_cast<const uint4*>(vrow);
-      const uint32_t vw[4] = {vb.x, vb.y, vb.z, vb.w};
-      uint32_t wv[8];
+  if (worker)
+    for (int rho = warp / S; rho < r; rho += P) {
+      float val = 0.f;
+      if (active) {
+        const uint4 vb = rho < rv ? *reinterpret_cast<const uint4*>(area + ap.vstage + (size_t)rho * (K / 8) + (size_t)g * 16)
+                                  : __ldg(reinterpret_cast<const uint4*>(it.vbits + (size_t)rho * (K / 32) + (size_t)g * 4));
+        const uint32_t vw[4] = {vb.x, vb.y, vb.z, vb.w};
+        uint32_t wv[8];
 #pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        const int wsw = hsw ? (w ^ 4) : w;  // limb registers are in swapped order on these lanes
-        wv[w] = spread16(~(vw[wsw >> 1] >> (16 * (wsw & 1))) & 0xFFFFu) << 1;
+        for (int w = 0; w < 8; ++w) {
+          const int wsw = hsw ? (w ^ 4) : w;  // limb registers are in swapped order on these lanes
+          wv[w] = spread16(~(vw[wsw >> 1] >> (16 * (wsw & 1))) & 0xFFFFu) << 1;
+        }
+        val = (float)(group_dot(wv, lb) - xs) * gsc;
       }
-      val = (float)(group_dot(wv, lb) - xs) * gsc;
+      val = warp_sum(val);
+      if (lane == 0) partz[W.s * WAL_MAX_RANK + rho] = val;
     }
-    val = warp_sum(val);
-    if (lane == 0) partz[s * WAL_MAX_RANK + rho] = val;
+  const uint32_t tab = ptx::smem_u32(area + ap.table) + (uint32_t)g * table_stride(SIGNED_TABLE) * 4u;
+  bool ok = true;
+  if (worker) {
+    switch (ks) {
+      case 8: ok = run_rows<8, SIGNED_TABLE>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
+      case 4: ok = run_rows<4, SIGNED_TABLE>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
+      case 2: ok = run_rows<2, SIGNED_TABLE>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
+      default: ok = run_rows<0, SIGNED_TABLE>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
+    }
   }
 
-  const uint32_t tab = smem_addr(table) + (uint32_t)g * 4u;
-  const uint32_t gs4 = Gp * 4u;
-  switch (ks) {
-    case 8: run_rows<8, SIGNED_TABLE>(W, RB, lane, active, hsw, lb, xs, gsc, tab, gs4, part, prm.status); break;
-    case 4: run_rows<4, SIGNED_TABLE>(W, RB, lane, active, hsw, lb, xs, gsc, tab, gs4, part, prm.status); break;
-    case 2: run_rows<2, SIGNED_TABLE>(W, RB, lane, active, hsw, lb, xs, gsc, tab, gs4, part, prm.status); break;
-    default: run_rows<0, SIGNED_TABLE>(W, RB, lane, active, hsw, lb, xs, gsc, tab, gs4, part, prm.status); break;
-  }
-  __syncthreads();
+  // after its own rows, warm L2 with the CTA's next tile
+  if (tid == 0)
+    for (int jn = j + 1; jn < R.n_groups; ++jn) {
+      const TileRec tn = R.sched[jn];
+      if (tn.rows) {
+        prefetch_tile(tn, R.items[tn.item]);
+        break;
+      }
+    }
 
-  // 4. slices and lanes in order, WALB2 phase 2, one store per output
+  const bool all_ok = !__syncthreads_or(!ok);
+
+  // slices and lanes in order, WALB2 phase 2, one store per output
   if (tid < r) {
     float a = 0.f;
     for (int s2 = 0; s2 < S; ++s2) a += partz[s2 * WAL_MAX_RANK + tid];
@@ -550,12 +646,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
   }
   __syncthreads();
   for (int rl = tid; rl < rows; rl += threads) {
-    const float* pr = part + (size_t)rl * 32;
+    const float* pr = part + (size_t)rl * kPartStride;
     float acc = 0.f;
     for (int s2 = 0; s2 < S; ++s2) {
       float a = 0.f;
 #pragma unroll
-      for (int l = 0; l < 32; ++l) a += pr[(size_t)s2 * RB * 32 + l];
+      for (int l = 0; l < 32; ++l) a += pr[(size_t)s2 * RB * kPartStride + l];
       acc += a;
     }
     if (r > 0) {
@@ -566,6 +662,96 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
     }
     it.y[n0 + rl] = acc;
   }
+  __syncthreads();  // the area is rebuilt by the next group
+  return all_ok;
+}
+
+// All CTAs of the launch meet here; `target` = CTAs x barriers passed so far.
+__device__ __forceinline__ void grid_barrier(unsigned int* ctr, unsigned int target, int32_t* status) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1u);
+    for (uint32_t it = 0; ld_acquire(ctr) < target; ++it)
+      if (it >= kBarrierSpin) {
+        if (status) atomicExch(status, (int32_t)WAL_ERR_TIMEOUT);
+        break;
+      }
+    __threadfence();
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_constant__ StreamParams prm) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ float s_z[WAL_MAX_RANK];
+  const bool table_mode = prm.t_sched != nullptr;
+  const StreamItem* items = table_mode ? prm.t_items : prm.items;
+  const int n_groups = table_mode ? prm.n_groups : 1;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, warps = (int)blockDim.x / 32;
+  const int stages = prm.stages;
+  if (!table_mode && blockIdx.x == 0 && tid == 0 && prm.status) *prm.status = 0;  // no timeout seen yet
+
+  // this CTA's schedule into shared memory
+  TileRec* sched = reinterpret_cast<TileRec*>(smem + prm.sched_off);
+  if (table_mode) {
+    const TileRec* src = prm.t_sched + (size_t)blockIdx.x * n_groups;
+    for (int jj = tid; jj < n_groups; jj += blockDim.x) sched[jj] = src[jj];
+  } else if (tid == 0) {
+    sched[0] = tile_record(prm.group, prm.items, blockIdx.x);
+  }
+  __syncthreads();
+
+  RingCtx R;
+  const uint32_t base = ptx::smem_u32(smem);
+  R.ring = base + (uint32_t)warp * stages * kChunkBytes;
+  R.mbar = base + ring_bytes(warps, stages) + (uint32_t)warp * stages * 8u;
+  R.ps = reinterpret_cast<ProdState*>(smem + ring_bytes(warps, stages) + (uint32_t)warps * stages * 8u +
+                                      (uint32_t)warp * (uint32_t)((sizeof(ProdState) + 15) & ~(size_t)15));
+  R.stages = stages;
+  R.sched = sched;
+  R.items = items;
+  R.n_groups = n_groups;
+  R.warp = warp;
+  R.items_global = table_mode;
+  R.status = prm.status;
+  if (lane == 0) {
+    for (int st = 0; st < stages; ++st) mbar_init(R.mbar + 8u * st, 1u);
+    ptx::mbar_init_fence();
+    R.ps->j = 0;
+    R.ps->issued = 0;
+    R.ps->consumed = 0;
+    prod_seek(*R.ps, sched, n_groups, items, warp);
+    for (int s0 = 0; s0 < stages; ++s0) prod_issue(*R.ps, R.ring, R.mbar, (uint32_t)s0, sched, n_groups, items, warp);
+  }
+  __syncwarp();
+
+  unsigned char* area = smem + prm.area_off;
+  uint32_t st = 0, parity = 0;  // this warp's ring slot and its phase parity
+  unsigned int nbar = 0;
+  bool dead = false;
+  for (int j = 0; j < n_groups; ++j) {
+    const TileRec t = sched[j];
+    if (j > 0 && t.stage != sched[j - 1].stage) {
+      ++nbar;
+      grid_barrier(prm.barrier, nbar * gridDim.x, prm.status);
+    }
+    if (t.rows == 0 || dead) continue;  // uniform across the CTA
+    const bool ok = t.signed_table ? do_group<true>(t, R, j, st, parity, area, s_z)
+                                   : do_group<false>(t, R, j, st, parity, area, s_z);
+    dead = !ok;
+  }
+  // never leave with bulk copies in flight: after a wait gave up, wait
+  // (bounded) for the chunks this warp issued but did not consume; they sit
+  // in consecutive slots from the current one
+  if (lane == 0 && dead)
+    for (uint32_t k = R.ps->consumed; k < R.ps->issued; ++k) {
+      if (!mbar_wait(R.mbar + st * 8u, parity, nullptr)) break;
+      if (++st == (uint32_t)stages) {
+        st = 0;
+        parity ^= 1u;
+      }
+    }
 }
 
 // ----------------------------------------------------------------------------
@@ -576,7 +762,6 @@ int g_sms = 0;
 int g_max_smem = 0;
 std::once_flag g_once;
 cudaError_t g_err = cudaSuccess;
-constexpr int kStageChoices[2] = {4, 2};
 }  // namespace
 
 int stream_init() {
@@ -585,11 +770,8 @@ int stream_init() {
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&g_max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    const int lim = g_max_smem - 1024;
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(stream_kernel<true, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(stream_kernel<false, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(stream_kernel<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(stream_kernel<false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, g_max_smem - 1024);
     g_err = e;
   });
   if (g_err != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("device initialisation: ") + cudaGetErrorString(g_err));
@@ -598,87 +780,119 @@ int stream_init() {
 
 int num_sms() { return g_sms > 0 ? g_sms : 148; }
 
-// Plan one launch over `n` products that share K.
-int plan_stream(const StreamItem* items, int n, int K, StreamLaunch* out) {
-  if (n < 1 || n > kMaxItems) return fail(WAL_ERR_ARG, "a stream launch takes 1..16 products");
-  StreamLaunch L;
-  L.S = (K + kSliceCols - 1) / kSliceCols;
-  if (L.S > kMaxThreads / 32) return fail(WAL_ERR_UNSUPPORTED, "K above 49152 is not handled by this build");
-  L.P = std::max(1, (kMaxThreads / 32) / L.S);
-  L.threads = 32 * L.S * L.P;
-  if (K / 8 > kMaxXChunks * L.threads) return fail(WAL_ERR_UNSUPPORTED, "K too large for the x-chunk registers");
+int plan_group(StreamItem* items, int n, int K, GroupDesc* out) {
+  if (n < 1 || n > kMaxItems) return fail(WAL_ERR_ARG, "a group takes 1..16 products");
+  GroupDesc g = {};
+  g.K = K;
+  g.S = (K + kSliceCols - 1) / kSliceCols;
+  if (g.S > kMaxWarps) return fail(WAL_ERR_UNSUPPORTED, "K above 49152 is not handled by this build");
+  g.P = std::max(1, kMaxWarps / g.S);
+  const int threads = 32 * g.S * g.P;
+  if (K / 8 > kMaxXChunks * threads) return fail(WAL_ERR_UNSUPPORTED, "K too large for the x-chunk registers");
   int rmax = 0;
-  long total_rows = 0;
-  for (int i = 0; i < n; ++i) {
-    rmax = std::max(rmax, items[i].r);
-    total_rows += items[i].N;
-  }
+  for (int i = 0; i < n; ++i) rmax = std::max(rmax, items[i].r);
+  g.rmax = rmax;
+  // smallest row block that keeps the group in one wave
   const int sms = num_sms();
-  // one tile per SM where possible: the smallest RB whose tile count fits one wave
-  int RB = (int)std::max(1L, (total_rows + sms - 1) / sms);
-  for (;;) {
-    long tiles = 0;
+  int total_rows = 0;
+  for (int i = 0; i < n; ++i) total_rows += items[i].N;
+  int RB = std::max(1, (total_rows + sms - 1) / sms);
+  for (;; ++RB) {
+    int tiles = 0;
     for (int i = 0; i < n; ++i) tiles += (items[i].N + RB - 1) / RB;
-    if (tiles <= sms || RB >= 4096) break;
-    ++RB;
+    if (tiles <= sms) break;
   }
-  L.RB = RB;
-  L.rmax = rmax;
-  // richest configuration that fits: deeper ring, +-X table, staged V planes
-  const int limit = g_max_smem - 1024;
-  bool found = false;
-  SmemPlan sp = {};
-  for (int trial = 0; trial < 8 && !found; ++trial) {
-    L.stages = kStageChoices[(trial >> 2) & 1];
-    L.signed_table = !(trial & 2);
-    L.stage_v = !(trial & 1) && rmax > 0;
-    sp = smem_plan(K, L.threads, L.S, L.RB, rmax, L.signed_table, L.stages, L.stage_v);
-    found = (int)sp.total <= limit;
+  if (RB > 65535) return fail(WAL_ERR_UNSUPPORTED, "row block above 65535 rows");
+  g.RB = RB;
+  int t = 0;
+  for (int i = 0; i < n; ++i) {
+    items[i].tile_begin = t;
+    t += (items[i].N + RB - 1) / RB;
   }
-  while (!found && L.RB > 1) {
-    L.RB = std::max(1, L.RB / 2);
-    sp = smem_plan(K, L.threads, L.S, L.RB, rmax, L.signed_table, L.stages, L.stage_v);
-    found = (int)sp.total <= limit;
-  }
-  if (!found) return fail(WAL_ERR_UNSUPPORTED, "K too large for the shared-memory plan");
-  L.smem = sp.total;
-  int tiles = 0;
-  for (int i = 0; i < n; ++i) tiles += (items[i].N + L.RB - 1) / L.RB;
-  L.tiles = tiles;
-  *out = L;
+  g.tiles = t;
+  g.n_items = n;
+  g.signed_table = 1;
+  *out = g;
   return WAL_OK;
 }
 
-int launch_stream(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream, bool pdl) {
-  prm.S = L.S;
-  prm.P = L.P;
-  prm.RB = L.RB;
-  prm.rmax = L.rmax;
-  prm.stage_v = L.stage_v ? 1 : 0;
-  int t = 0;
-  for (int i = 0; i < prm.n_items; ++i) {
-    prm.items[i].tile_begin = t;
-    t += (prm.items[i].N + L.RB - 1) / L.RB;
+int plan_launch(GroupDesc* groups, int n_groups, bool persistent, StreamLaunch* out) {
+  StreamLaunch L = {};
+  int warps = 0;
+  for (int j = 0; j < n_groups; ++j) warps = std::max(warps, groups[j].S * groups[j].P);
+  if (persistent) warps = kMaxWarps;
+  L.threads = 32 * warps;
+  const uint32_t limit = (uint32_t)(g_max_smem > 0 ? g_max_smem : 232448) - 1024u;
+  const uint32_t sched_bytes = (uint32_t)align_up((size_t)n_groups * sizeof(TileRec), 128);
+  for (int stages : {4, 3, 2}) {
+    const uint32_t soff = area_offset(warps, stages);
+    const uint32_t off = soff + sched_bytes;
+    uint32_t need = off;
+    bool fits = true;
+    for (int j = 0; j < n_groups && fits; ++j) {
+      const GroupDesc& g = groups[j];
+      const uint32_t as = area_plan(g.K, g.S, g.RB, true).total, au = area_plan(g.K, g.S, g.RB, false).total;
+      if (off + as <= limit) need = std::max(need, off + as);
+      else if (off + au <= limit) need = std::max(need, off + au);
+      else fits = false;
+    }
+    if (!fits) continue;
+    for (int j = 0; j < n_groups; ++j) {
+      const GroupDesc& g = groups[j];
+      groups[j].signed_table = off + area_plan(g.K, g.S, g.RB, true).total <= limit ? 1 : 0;
+    }
+    L.stages = stages;
+    L.sched_off = soff;
+    L.area_off = off;
+    L.smem = need;
+    int tiles = 0;
+    for (int j = 0; j < n_groups; ++j) tiles = std::max(tiles, groups[j].tiles);
+    L.grid = persistent ? num_sms() : tiles;
+    *out = L;
+    return WAL_OK;
   }
+  return fail(WAL_ERR_UNSUPPORTED, "K too large for the shared-memory plan");
+}
+
+void build_schedule(const GroupDesc* groups, int n_groups, const StreamItem* items, int cta, TileRec* out) {
+  for (int j = 0; j < n_groups; ++j) out[j] = tile_record(groups[j], items + groups[j].item0, cta);
+}
+
+static int launch(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream, bool cooperative) {
+  prm.stages = L.stages;
+  prm.sched_off = L.sched_off;
+  prm.area_off = L.area_off;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(L.tiles);
+  cfg.gridDim = dim3(L.grid);
   cfg.blockDim = dim3(L.threads);
   cfg.dynamicSmemBytes = L.smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  cudaError_t e;
-  if (L.stages == 4)
-    e = L.signed_table ? cudaLaunchKernelEx(&cfg, stream_kernel<true, 4>, prm)
-                       : cudaLaunchKernelEx(&cfg, stream_kernel<false, 4>, prm);
-  else
-    e = L.signed_table ? cudaLaunchKernelEx(&cfg, stream_kernel<true, 2>, prm)
-                       : cudaLaunchKernelEx(&cfg, stream_kernel<false, 2>, prm);
+  cfg.numAttrs = cooperative ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, stream_kernel, prm);
   if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("stream_kernel launch: ") + cudaGetErrorString(e));
   return WAL_OK;
+}
+
+int launch_stream(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream) {
+  prm.t_sched = nullptr;
+  prm.t_items = nullptr;
+  prm.n_groups = 1;
+  prm.barrier = nullptr;
+  return launch(prm, L, stream, false);
+}
+
+int launch_body(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream) {
+  if (!prm.t_sched || !prm.t_items || !prm.barrier) return fail(WAL_ERR_ARG, "body launch without tables");
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, stream_kernel, L.threads, L.smem);
+  if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("occupancy query: ") + cudaGetErrorString(e));
+  if (per_sm < 1 || L.grid > per_sm * num_sms())
+    return fail(WAL_ERR_UNSUPPORTED, "the persistent launch does not fit on the device at once");
+  return launch(prm, L, stream, true);
 }
 
 }  // namespace wal

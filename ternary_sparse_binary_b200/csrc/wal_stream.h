@@ -8,9 +8,8 @@
 namespace wal {
 
 constexpr int kMaxItems = 16;
-constexpr int kMaxPrefetch = 24;
 
-// One product y = W x inside a launch.
+// One product y = W x.
 struct StreamItem {
   const uint32_t* codes;
   const uint8_t* sites;
@@ -21,32 +20,63 @@ struct StreamItem {
   const uint16_t* x;  // bf16 [K]
   float* y;           // fp32 [N]
   int N, k, r;
-  int tile_begin;     // first tile of this product (filled by launch_stream)
+  int tile_begin;     // first tile of this product inside its group
 };
 
-// A byte range to warm in L2 (16-byte aligned start, size a multiple of 16).
-struct PrefetchRange {
-  const void* ptr;
-  unsigned long long bytes;
+// A group: up to 16 products that share K and run together, one tile of RB
+// rows per CTA.  Groups of one dependency stage run back to back; between
+// stages the CTAs meet at a grid barrier.
+struct GroupDesc {
+  int K, S, P, RB, rmax, tiles;
+  int signed_table;  // +-X table (256 entries) or X table with the sign applied at lookup
+  int item0, n_items;
+  int stage;         // dependency stage (non-decreasing along the group list)
 };
 
+// What one CTA does in one group (16 bytes; a body pass keeps [CTA][group]
+// of these in device memory and each CTA copies its row into shared memory).
+struct TileRec {
+  uint16_t item;   // index into the item table
+  uint16_t rows;   // rows of the tile (0: the CTA has no tile in this group)
+  int32_t n0;      // first output row of the tile
+  uint8_t G, S, P, signed_table;  // K / 128, slices, phases, table kind
+  uint16_t RB;     // rows per tile of the group
+  uint16_t stage;  // dependency stage
+};
+
+// Parameters of one launch: either one inline group (a single product call)
+// or per-CTA schedules and an item table in device memory (a body pass).
 struct StreamParams {
   StreamItem items[kMaxItems];
-  PrefetchRange pf[kMaxPrefetch];
-  int n_items, n_pf;
-  int K, S, P, RB, rmax, stage_v;
-  int32_t* status;  // workspace status word, cleared by the launch (may be NULL)
+  GroupDesc group;
+  const TileRec* t_sched;     // NULL: use the inline group; else [gridDim.x][n_groups]
+  const StreamItem* t_items;
+  int n_groups;
+  int stages;                 // ring depth (rows per warp = 2 * stages)
+  uint32_t sched_off;         // shared-memory offset of the CTA's schedule
+  uint32_t area_off;          // shared-memory offset of the per-group area
+  unsigned int* barrier;      // grid-barrier counter (zeroed before the launch), body pass only
+  int32_t* status;            // workspace status word (may be NULL)
 };
 
 struct StreamLaunch {
-  int S, P, RB, threads, tiles, rmax, stages;
-  bool signed_table, stage_v;
+  int grid, threads, stages;
   unsigned smem;
+  uint32_t sched_off, area_off;
 };
+
+// The schedule row of CTA `cta` for groups[0 .. n_groups) (items as planned).
+void build_schedule(const GroupDesc* groups, int n_groups, const StreamItem* items, int cta, TileRec* out);
 
 int stream_init();
 int num_sms();
-int plan_stream(const StreamItem* items, int n, int K, StreamLaunch* out);
-int launch_stream(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream, bool pdl);
+// Fill the geometry of group `g` (K, items) and return WAL_OK or an error.
+int plan_group(StreamItem* items, int n, int K, GroupDesc* g);
+// Shared memory and ring depth for a list of groups.
+int plan_launch(GroupDesc* groups, int n_groups, bool persistent, StreamLaunch* out);
+// Single group, items inline.
+int launch_stream(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream);
+// Body pass: group and item tables already in device memory; cooperative launch.
+int launch_body(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream);
 
 }  // namespace wal

@@ -4,31 +4,36 @@ import pytest
 import torch
 
 import oracle
-from wal_synth import config_plan, gen_matrix, gen_x, body_plan, LAYER_8B
+from wal_synth import config_plan, gen_components, gen_matrix, gen_x, body_plan, bf16_bits_from_f32, LAYER_8B
 
 from gpu_util import needs_gpu, wal, device_matrix, device_bf16, assert_parity
 
 pytestmark = [pytest.mark.gpu, needs_gpu]
 
 
-def _run_plan(workload, specs, sample=64, replays=2):
+def _status(bp):
+    wal().wal_device_status(bp.ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+
+
+def _run_plan(workload, specs, sample=64, replays=2, M=1):
     w = wal()
     mats, xs, ys, comps, xbits = [], [], [], [], []
     for s in specs:
         c = gen_matrix(workload, s)
-        x = gen_x(s.K, 1, 2 if workload == "body8b" else 1, s.index)
+        x = gen_x(s.K, M, 2 if workload == "body8b" else 1, s.index)
         mats.append(device_matrix(c))
         xs.append(device_bf16(x))
-        ys.append(torch.empty(s.N, dtype=torch.float32, device="cuda"))
+        ys.append(torch.empty((M, s.N), dtype=torch.float32, device="cuda"))
         comps.append(c if sample else None)
-        xbits.append(x[0])
-    bp = w.BodyPass(mats, [s.stage for s in specs], xs, ys, M=1)
+        xbits.append(x)
+    bp = w.BodyPass(mats, [s.stage for s in specs], xs, ys, M=M)
     outs = []
     for _ in range(replays):
         for y in ys:
             y.fill_(float("nan"))
         bp.run()
         torch.cuda.synchronize()
+        _status(bp)
         outs.append([y.cpu().numpy().astype(np.float64) for y in ys])
     bp.close()
     return specs, comps, xbits, outs
@@ -41,7 +46,55 @@ def test_body_two_layers_sampled():
     for s, c, x, y, y2 in zip(specs, comps, xbits, outs[0], outs[1]):
         assert np.array_equal(y, y2), "graph replays differ"
         rows = np.unique(np.concatenate([[0, s.N - 1], rng.choice(s.N, 64, replace=False)]))
-        assert_parity(y[rows], oracle.matmul_rows(c, x, rows)[0], x, c.alpha, s.name)
+        assert_parity(y[0][rows], oracle.matmul_rows(c, x, rows)[0], x, c.alpha, s.name)
+
+
+def test_body_batch4_two_layers():
+    """M = 4: four activation rows per matrix in one pass."""
+    specs = body_plan(2, LAYER_8B, 8, 8, 1, n_lowrank=9)
+    specs, comps, xbits, outs = _run_plan("layer8b", specs, replays=1, M=4)
+    rng = np.random.default_rng(13)
+    for s, c, X, Y in zip(specs, comps, xbits, outs[0]):
+        rows = np.unique(rng.choice(s.N, 48, replace=False))
+        assert_parity(Y[:, rows], oracle.matmul_rows(c, X, rows), X, c.alpha, s.name)
+
+
+def test_body_stage_dependency():
+    """Stage 1 reads what stage 0 writes.  Stage 0 is a selection matrix
+    (y_A[n] = x_A[n mod K_A], alpha = 1), so its fp32 outputs are bf16 values
+    exactly; read as bf16 pairs, y_A's bytes are (0, y_A[n]) for every n.
+    Matrix B of stage 1 takes that buffer as its x.  The buffer starts as
+    NaN, so a read before the grid barrier shows."""
+    w = wal()
+    NA, KA = 2048, 1024
+    a = gen_components(NA, KA, 0, 0, config_id=60, matrix_index=0)
+    a.T[:] = 0
+    a.T[np.arange(NA), np.arange(NA) % KA] = 1
+    a.alpha[:] = 0x3C00  # fp16 1.0
+    # magnitudes in [1, 2): every x_A is exact in the fixed-point image, so
+    # y_A holds bf16 values exactly
+    rng = np.random.default_rng(60)
+    xa = bf16_bits_from_f32((rng.uniform(1.0, 2.0, (1, KA)) * rng.choice([-1.0, 1.0], (1, KA))).astype(np.float32))
+    b = gen_components(4096, 2 * NA, 8, 8, config_id=60, matrix_index=1)
+    c2 = gen_components(1024, 4096, 4, 0, config_id=60, matrix_index=2)  # a second stage-1 matrix, own x
+    xc = gen_x(4096, 1, 60, 2)
+    ya = torch.full((NA,), float("nan"), dtype=torch.float32, device="cuda")
+    xb = ya.view(torch.int16)  # the same bytes as 2 * NA bf16 values
+    yb = torch.empty(4096, dtype=torch.float32, device="cuda")
+    yc = torch.empty(1024, dtype=torch.float32, device="cuda")
+    mats = [device_matrix(a), device_matrix(b), device_matrix(c2)]
+    bp = w.BodyPass(mats, [0, 1, 1], [device_bf16(xa), xb, device_bf16(xc)], [ya, yb, yc], M=1)
+    for _ in range(2):
+        ya.fill_(float("nan"))
+        bp.run()
+        torch.cuda.synchronize()
+        _status(bp)
+        exp_a = oracle.matvec(a, xa[0])
+        assert np.array_equal(ya.cpu().numpy().astype(np.float64), exp_a)
+        xb_bits = ya.cpu().numpy().view(np.uint16)
+        assert_parity(yb.cpu().numpy().astype(np.float64), oracle.matvec(b, xb_bits), xb_bits, b.alpha, "stage 1")
+        assert_parity(yc.cpu().numpy().astype(np.float64), oracle.matvec(c2, xc[0]), xc[0], c2.alpha, "stage 1 other")
+    bp.close()
 
 
 def test_body8b_full_sampled():
@@ -64,6 +117,7 @@ def test_body8b_full_sampled():
     bp = w.BodyPass(mats, [s.stage for s in specs], xs, ys, M=1)
     bp.run()
     torch.cuda.synchronize()
+    _status(bp)
     for (s, rows, ref, x, alpha), y in zip(checks, ys):
         assert_parity(y.cpu().numpy().astype(np.float64)[rows], ref, x, alpha, s.name)
     bp.close()
