@@ -38,9 +38,10 @@
 //    (exact).  alpha and beta are applied in FP32 and the group weight once.
 //    The WALB2 phase-1 products V_r^T x go through the same path: a row of
 //    V is a ternary row without zeros, its bits spread into 2-bit codes.
-//  - Each lane leaves its group's partial in shared memory; after the rows
-//    one thread per output row sums the slices and lanes in a fixed order,
-//    and the WALB2 phase-2 term sum_r U[n, r] z_r joins in the single store.
+//  - Each row's lane partials are summed across the warp by a fixed
+//    butterfly; after the rows one thread per output row adds the slices in
+//    order, and the WALB2 phase-2 term sum_r U[n, r] z_r joins in the single
+//    store.
 // Results are bitwise reproducible: no atomics in the arithmetic, fixed
 // reduction orders.  Every wait (mbarrier, grid barrier) is bounded; one that
 // gives up records WAL_ERR_TIMEOUT in the status word and the waiter moves on.
@@ -60,24 +61,32 @@ using ptx::mbar_arrive_expect_tx;
 using ptx::mbar_wait;
 using ptx::bulk_g2s;
 
-constexpr int kRowsPerStage = 3;  // rows per ring chunk
+constexpr int kMaxRowsPerChunk = 3;  // rows per ring chunk: 3, or 2 where shared memory is short
 constexpr int kMaxThreads = 384;
 constexpr int kMaxWarps = kMaxThreads / 32;
 constexpr int kMaxXChunks = 8;            // 8-column chunks of x per thread
 constexpr uint32_t kMagic = 0x4B400000u;  // 1.5 * 2^23: adding it rounds |v| < 2^22 to an integer
 constexpr uint32_t kLimbStride = 100;     // words per group in the limb image (96 + 4 pad)
-constexpr uint32_t kPartStride = 33;      // floats per row of per-lane partials (32 + 1 pad: the combine reads a row per thread)
 constexpr uint32_t kBarrierSpin = 1u << 22;  // polls of the grid-barrier counter before giving up
-// One ring chunk of one warp: three rows of codes (32 lanes x 32 B each), then
+// One ring chunk of one warp: rpc rows of codes (32 lanes x 32 B each), then
 // their site bytes (32 x 8 B each + 16 B alignment slack), then their
 // {alpha, beta} words (32 x 4 B each + 16 B slack).  With a single K-slice
-// (K <= 4096) the three rows are contiguous in every buffer and arrive as one
-// copy per buffer, packed at the buffers' own row pitch; otherwise each row is
+// (K <= 4096) the rows are contiguous in every buffer and arrive as one copy
+// per buffer, packed at the buffers' own row pitch; otherwise each row is
 // copied on its own at the fixed pitches below.
 constexpr uint32_t kCodePitch = 1024, kSitePitch = 272, kScalePitch = 144;
-constexpr uint32_t kChunkSites = kRowsPerStage * kCodePitch;
-constexpr uint32_t kChunkScales = kChunkSites + kRowsPerStage * kSitePitch;
-constexpr uint32_t kChunkBytes = kChunkScales + kRowsPerStage * kScalePitch;
+struct ChunkGeom {
+  int rpc;                        // rows per chunk
+  uint32_t sites, scales, bytes;  // offsets of the site and scale parts, chunk size
+};
+__host__ __device__ inline ChunkGeom chunk_geom(int rpc) {
+  ChunkGeom c;
+  c.rpc = rpc;
+  c.sites = (uint32_t)rpc * kCodePitch;
+  c.scales = c.sites + (uint32_t)rpc * kSitePitch;
+  c.bytes = c.scales + (uint32_t)rpc * kScalePitch;
+  return c;
+}
 
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
@@ -153,26 +162,24 @@ __device__ __forceinline__ int32_t group_dot(const uint32_t (&wv)[8], const uint
 // that groups land on different banks.
 __host__ __device__ inline uint32_t table_stride(bool signed_table) { return signed_table ? 257u : 129u; }
 
-__host__ __device__ inline uint32_t ring_bytes(int warps, int stages) {
-  return (uint32_t)warps * stages * kChunkBytes;
+__host__ __device__ inline uint32_t ring_bytes(int warps, int stages, int rpc) {
+  return (uint32_t)warps * stages * chunk_geom(rpc).bytes;
 }
 struct ProdState;  // defined below
-__host__ __device__ inline uint32_t area_offset(int warps, int stages);
+__host__ __device__ inline uint32_t area_offset(int warps, int stages, int rpc);
 
 struct AreaPlan {
   uint32_t table, limbs, part, xgsum, gsc, partz, ubuf, vstage, total;
 };
-// Carve-up of the per-group area (offsets relative to the area base).  The
-// limb image is dead once every warp holds its limbs in registers; the
-// per-lane partials, written only after that, reuse its space.
+// Carve-up of the per-group area (offsets relative to the area base).
 __host__ __device__ inline AreaPlan area_plan(int K, int S, int RB, bool signed_table) {
   AreaPlan p;
   uint32_t off = 0;
   auto take = [&](uint32_t bytes) { uint32_t o = off; off = (off + bytes + 15u) & ~15u; return o; };
   const uint32_t G = (uint32_t)K / kGroup;
   p.table = take(G * table_stride(signed_table) * 4u);
-  const uint32_t limbs = G * kLimbStride * 4u, part = (uint32_t)S * RB * kPartStride * 4u;
-  p.limbs = p.part = take(part > limbs ? part : limbs);
+  p.limbs = take(G * kLimbStride * 4u);
+  p.part = take((uint32_t)S * RB * 4u);  // one partial per (slice, row)
   p.xgsum = take(G * 4u);
   p.gsc = take(G * 4u);
   p.partz = take((uint32_t)S * WAL_MAX_RANK * 4u);
@@ -238,9 +245,10 @@ __device__ __forceinline__ uint32_t scale_bytes(int k) { return k > 0 ? 4u : 2u;
 // `bar`.  Site and scale ranges are widened to 16-byte boundaries (every
 // buffer is zero-padded to a multiple of 16 bytes, so the widened range stays
 // inside).
-__device__ __forceinline__ void issue_chunk(const WarpRing& W, uint32_t sl, uint32_t bar, int chunk) {
-  const int i0 = chunk * kRowsPerStage;
-  const int un = min(kRowsPerStage, W.nmine - i0);
+__device__ __forceinline__ void issue_chunk(const WarpRing& W, uint32_t sl, uint32_t bar, int chunk,
+                                            const ChunkGeom& C) {
+  const int i0 = chunk * C.rpc;
+  const int un = min(C.rpc, W.nmine - i0);
   if (un <= 0) return;
   const uint32_t kb = site_bytes(W.k), sb = scale_bytes(W.k);
   const unsigned char* cbase = reinterpret_cast<const unsigned char*>(W.codes);
@@ -252,8 +260,8 @@ __device__ __forceinline__ void issue_chunk(const WarpRing& W, uint32_t sl, uint
     const size_t aa = (n * G * sb) & ~(size_t)15, ae = ((n + un) * G * sb + 15) & ~(size_t)15;
     mbar_arrive_expect_tx(bar, clen + (uint32_t)(se - sa) + (uint32_t)(ae - aa));
     bulk_g2s(sl, cbase + n * (size_t)(W.K / 4), clen, bar);
-    if (se > sa) bulk_g2s(sl + kChunkSites, W.sites + sa, (uint32_t)(se - sa), bar);
-    bulk_g2s(sl + kChunkScales, abase + aa, (uint32_t)(ae - aa), bar);
+    if (se > sa) bulk_g2s(sl + C.sites, W.sites + sa, (uint32_t)(se - sa), bar);
+    bulk_g2s(sl + C.scales, abase + aa, (uint32_t)(ae - aa), bar);
     return;
   }
   // several K-slices: each row on its own (lengths first for the expected bytes)
@@ -282,8 +290,8 @@ __device__ __forceinline__ void issue_chunk(const WarpRing& W, uint32_t sl, uint
     site_range(gb, a, e);
     scale_range(gb, a2, e2);
     bulk_g2s(sl + (uint32_t)u * kCodePitch, cbase + n * (size_t)(W.K / 4) + (size_t)W.s * 1024, (uint32_t)ng * 32u, bar);
-    if (e > a) bulk_g2s(sl + kChunkSites + (uint32_t)u * kSitePitch, W.sites + a, (uint32_t)(e - a), bar);
-    bulk_g2s(sl + kChunkScales + (uint32_t)u * kScalePitch, abase + a2, (uint32_t)(e2 - a2), bar);
+    if (e > a) bulk_g2s(sl + C.sites + (uint32_t)u * kSitePitch, W.sites + a, (uint32_t)(e - a), bar);
+    bulk_g2s(sl + C.scales + (uint32_t)u * kScalePitch, abase + a2, (uint32_t)(e2 - a2), bar);
   }
 }
 
@@ -295,20 +303,20 @@ struct ProdState {
   uint32_t consumed;  // chunks consumed so far
   WarpRing W;
 };
-__host__ __device__ inline uint32_t area_offset(int warps, int stages) {
-  const uint32_t o = ring_bytes(warps, stages) + (uint32_t)warps * stages * 8u +
+__host__ __device__ inline uint32_t area_offset(int warps, int stages, int rpc) {
+  const uint32_t o = ring_bytes(warps, stages, rpc) + (uint32_t)warps * stages * 8u +
                      (uint32_t)warps * (uint32_t)((sizeof(ProdState) + 15) & ~(size_t)15);
   return (o + 127u) & ~127u;
 }
 
 // Move the producer to the first group at or after ps.j with rows for this warp.
 __device__ __forceinline__ void prod_seek(ProdState& ps, const TileRec* sched, int n_groups, const StreamItem* items,
-                                          int warp) {
+                                          int warp, int rpc) {
   while (ps.j < n_groups) {
     const TileRec t = sched[ps.j];
     if (t.rows && warp < (int)t.S * t.P) {
       warp_work(t, items + t.item, warp, ps.W);
-      ps.nc = (ps.W.nmine + kRowsPerStage - 1) / kRowsPerStage;
+      ps.nc = (ps.W.nmine + rpc - 1) / rpc;
       ps.c = 0;
       if (ps.nc > 0) return;
     }
@@ -318,13 +326,14 @@ __device__ __forceinline__ void prod_seek(ProdState& ps, const TileRec* sched, i
 
 // Issue the producer's next chunk into ring slot st (if any is left).
 __device__ __forceinline__ void prod_issue(ProdState& ps, uint32_t ring, uint32_t mbar, uint32_t st,
-                                           const TileRec* sched, int n_groups, const StreamItem* items, int warp) {
+                                           const TileRec* sched, int n_groups, const StreamItem* items, int warp,
+                                           const ChunkGeom& C) {
   if (ps.j >= n_groups) return;
-  issue_chunk(ps.W, ring + st * kChunkBytes, mbar + st * 8u, ps.c);
+  issue_chunk(ps.W, ring + st * C.bytes, mbar + st * 8u, ps.c, C);
   ++ps.issued;
   if (++ps.c == ps.nc) {
     ++ps.j;
-    prod_seek(ps, sched, n_groups, items, warp);
+    prod_seek(ps, sched, n_groups, items, warp, C.rpc);
   }
 }
 
@@ -382,6 +391,7 @@ struct RingCtx {
   const TileRec* sched; // this CTA's schedule (shared memory)
   const StreamItem* items;
   int n_groups, warp;
+  ChunkGeom C;          // ring chunk geometry
   bool items_global;    // items live in device memory (not kernel parameters)
   int32_t* status;
 };
@@ -393,8 +403,9 @@ template <int KS, bool SIGNED_TABLE>
 __device__ __forceinline__ bool run_rows(const WarpRing& W, const RingCtx& R, uint32_t& st, uint32_t& parity, int RB,
                                          int lane, bool active, uint32_t hsw, const uint32_t (&lb)[8][kLimbWords],
                                          int32_t xs, float gsc, uint32_t tab, float* part) {
-  const int nc = (W.nmine + kRowsPerStage - 1) / kRowsPerStage;
-  float* mine = part + (W.s * RB + W.r0) * (int)kPartStride + lane;  // row i at mine[i * kPartStride]
+  const ChunkGeom& C = R.C;
+  const int nc = (W.nmine + C.rpc - 1) / C.rpc;
+  float* mine = part + W.s * RB + W.r0;  // this warp's row i at mine[i]
   const uint32_t kb = site_bytes(KS), sb = scale_bytes(KS);
   const bool one = W.one_slice();
   const uint32_t G = (uint32_t)W.G;
@@ -402,26 +413,27 @@ __device__ __forceinline__ bool run_rows(const WarpRing& W, const RingCtx& R, ui
   const uint32_t cp = one ? G * 32u : kCodePitch, sp = one ? G * kb : kSitePitch, ap = one ? G * sb : kScalePitch;
 #pragma unroll 1
   for (int j = 0; j < nc; ++j) {
-    const uint32_t sl = R.ring + st * kChunkBytes;
+    const uint32_t sl = R.ring + st * C.bytes;
     if (!mbar_wait(R.mbar + st * 8u, parity, R.status)) return false;
     // group index of the chunk's first row (this slice's first group)
-    const uint32_t gb0 = (uint32_t)(W.nb + j * kRowsPerStage) * G + 32u * (uint32_t)W.s;
+    const uint32_t gb0 = (uint32_t)(W.nb + j * C.rpc) * G + 32u * (uint32_t)W.s;
 #pragma unroll
-    for (int u = 0; u < kRowsPerStage; ++u) {
-      const int i = j * kRowsPerStage + u;
-      if (i < W.nmine) {  // uniform across the warp
+    for (int u = 0; u < kMaxRowsPerChunk; ++u) {
+      const int i = j * C.rpc + u;
+      if (u < C.rpc && i < W.nmine) {  // uniform across the warp
         const uint32_t gb = one ? gb0 : gb0 + (uint32_t)u * G;
-        const uint32_t srow = sl + kChunkSites + (uint32_t)u * sp + ((gb * kb) & 15u);
-        const uint32_t arow = sl + kChunkScales + (uint32_t)u * ap + ((gb * sb) & 15u);
+        const uint32_t srow = sl + C.sites + (uint32_t)u * sp + ((gb * kb) & 15u);
+        const uint32_t arow = sl + C.scales + (uint32_t)u * ap + ((gb * sb) & 15u);
         const float v =
             row_value<KS, SIGNED_TABLE>(sl + (uint32_t)u * cp, srow, arow, lane, hsw, lb, xs, gsc, tab);
-        mine[i * (int)kPartStride] = active ? v : 0.f;
+        const float tot = warp_sum(active ? v : 0.f);  // fixed butterfly order: reproducible
+        if (lane == 0) mine[i] = tot;
       }
     }
     __syncwarp();  // every lane has consumed the slot before it is refilled
     if (lane == 0) {
       ++R.ps->consumed;
-      prod_issue(*R.ps, R.ring, R.mbar, st, R.sched, R.n_groups, R.items, R.warp);
+      prod_issue(*R.ps, R.ring, R.mbar, st, R.sched, R.n_groups, R.items, R.warp, C);
     }
     if (++st == (uint32_t)R.stages) {
       st = 0;
@@ -595,7 +607,7 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
   }
 
   cp_async_wait<0>();
-  __syncthreads();  // staged U / V complete; the partials below overwrite the limb image
+  __syncthreads();  // staged U / V complete
   // WALB2 phase 1: rows of V (no zeros: bit set -> code 0, clear -> code 2)
   if (worker)
     for (int rho = warp / S; rho < r; rho += P) {
@@ -638,7 +650,7 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
 
   const bool all_ok = !__syncthreads_or(!ok);
 
-  // slices and lanes in order, WALB2 phase 2, one store per output
+  // slices in order, WALB2 phase 2, one store per output
   if (tid < r) {
     float a = 0.f;
     for (int s2 = 0; s2 < S; ++s2) a += partz[s2 * WAL_MAX_RANK + tid];
@@ -646,14 +658,8 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
   }
   __syncthreads();
   for (int rl = tid; rl < rows; rl += threads) {
-    const float* pr = part + (size_t)rl * kPartStride;
     float acc = 0.f;
-    for (int s2 = 0; s2 < S; ++s2) {
-      float a = 0.f;
-#pragma unroll
-      for (int l = 0; l < 32; ++l) a += pr[(size_t)s2 * RB * kPartStride + l];
-      acc += a;
-    }
+    for (int s2 = 0; s2 < S; ++s2) acc += part[s2 * RB + rl];
     if (r > 0) {
       const uint32_t uw = ubuf[rl];
       float lr = 0.f;
@@ -704,9 +710,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
 
   RingCtx R;
   const uint32_t base = ptx::smem_u32(smem);
-  R.ring = base + (uint32_t)warp * stages * kChunkBytes;
-  R.mbar = base + ring_bytes(warps, stages) + (uint32_t)warp * stages * 8u;
-  R.ps = reinterpret_cast<ProdState*>(smem + ring_bytes(warps, stages) + (uint32_t)warps * stages * 8u +
+  R.C = chunk_geom(prm.rpc);
+  R.ring = base + (uint32_t)warp * stages * R.C.bytes;
+  R.mbar = base + ring_bytes(warps, stages, prm.rpc) + (uint32_t)warp * stages * 8u;
+  R.ps = reinterpret_cast<ProdState*>(smem + ring_bytes(warps, stages, prm.rpc) + (uint32_t)warps * stages * 8u +
                                       (uint32_t)warp * (uint32_t)((sizeof(ProdState) + 15) & ~(size_t)15));
   R.stages = stages;
   R.sched = sched;
@@ -721,8 +728,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
     R.ps->j = 0;
     R.ps->issued = 0;
     R.ps->consumed = 0;
-    prod_seek(*R.ps, sched, n_groups, items, warp);
-    for (int s0 = 0; s0 < stages; ++s0) prod_issue(*R.ps, R.ring, R.mbar, (uint32_t)s0, sched, n_groups, items, warp);
+    prod_seek(*R.ps, sched, n_groups, items, warp, R.C.rpc);
+    for (int s0 = 0; s0 < stages; ++s0)
+      prod_issue(*R.ps, R.ring, R.mbar, (uint32_t)s0, sched, n_groups, items, warp, R.C);
   }
   __syncwarp();
 
@@ -824,8 +832,11 @@ int plan_launch(GroupDesc* groups, int n_groups, bool persistent, StreamLaunch* 
   L.threads = 32 * warps;
   const uint32_t limit = (uint32_t)(g_max_smem > 0 ? g_max_smem : 232448) - 1024u;
   const uint32_t sched_bytes = (uint32_t)align_up((size_t)n_groups * sizeof(TileRec), 128);
-  for (int stages : {4, 3, 2}) {
-    const uint32_t soff = area_offset(warps, stages);
+  // deepest ring first (rows in flight per warp), fewer copies on a tie
+  static const int kRing[6][2] = {{3, 4}, {3, 3}, {2, 4}, {3, 2}, {2, 3}, {2, 2}};
+  for (const auto& rs : kRing) {
+    const int rpc = rs[0], stages = rs[1];
+    const uint32_t soff = area_offset(warps, stages, rpc);
     const uint32_t off = soff + sched_bytes;
     uint32_t need = off;
     bool fits = true;
@@ -842,6 +853,7 @@ int plan_launch(GroupDesc* groups, int n_groups, bool persistent, StreamLaunch* 
       groups[j].signed_table = off + area_plan(g.K, g.S, g.RB, true).total <= limit ? 1 : 0;
     }
     L.stages = stages;
+    L.rpc = rpc;
     L.sched_off = soff;
     L.area_off = off;
     L.smem = need;
@@ -860,6 +872,7 @@ void build_schedule(const GroupDesc* groups, int n_groups, const StreamItem* ite
 
 static int launch(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream, bool cooperative) {
   prm.stages = L.stages;
+  prm.rpc = L.rpc;
   prm.sched_off = L.sched_off;
   prm.area_off = L.area_off;
   cudaLaunchConfig_t cfg = {};

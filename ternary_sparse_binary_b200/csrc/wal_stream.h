@@ -52,7 +52,8 @@ struct StreamParams {
   const TileRec* t_sched;     // NULL: use the inline group; else [gridDim.x][n_groups]
   const StreamItem* t_items;
   int n_groups;
-  int stages;                 // ring depth (rows per warp = 2 * stages)
+  int stages;                 // ring depth in chunks
+  int rpc;                    // rows per ring chunk (2 or 3)
   uint32_t sched_off;         // shared-memory offset of the CTA's schedule
   uint32_t area_off;          // shared-memory offset of the per-group area
   unsigned int* barrier;      // grid-barrier counter (zeroed before the launch), body pass only
@@ -60,7 +61,7 @@ struct StreamParams {
 };
 
 struct StreamLaunch {
-  int grid, threads, stages;
+  int grid, threads, stages, rpc;
   unsigned smem;
   uint32_t sched_off, area_off;
 };

@@ -121,3 +121,41 @@ def test_body8b_full_sampled():
     for (s, rows, ref, x, alpha), y in zip(checks, ys):
         assert_parity(y.cpu().numpy().astype(np.float64)[rows], ref, x, alpha, s.name)
     bp.close()
+
+
+@pytest.fixture(scope="module")
+def body27b():
+    """The 448 27B-shaped matrices on the device, with oracle values of 24
+    sampled rows of every matrix for x at M = 1 and M = 4."""
+    specs = config_plan("body27b")
+    rng = np.random.default_rng(27)
+    mats, checks = [], []
+    for s in specs:
+        c = gen_matrix("body27b", s)
+        rows = np.unique(rng.choice(s.N, 24, replace=False))
+        per_m = {}
+        for M in (1, 4):
+            X = gen_x(s.K, M, 3, 1000 * M + s.index)
+            per_m[M] = (X, oracle.matmul_rows(c, X, rows))
+        checks.append((s, rows, per_m, c.alpha.copy()))
+        mats.append(device_matrix(c))
+        del c
+    return specs, mats, checks
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_body27b_full_sampled(body27b, M):
+    """The full 448-matrix 27B-shaped body pass (k by role, 45 matrices with
+    k = 0, 152 with WALB2 r = 8) at batch 1 and 4."""
+    w = wal()
+    specs, mats, checks = body27b
+    xs = [device_bf16(per_m[M][0]) for (_, _, per_m, _) in checks]
+    ys = [torch.full((M, s.N), float("nan"), dtype=torch.float32, device="cuda") for s in specs]
+    bp = w.BodyPass(mats, [s.stage for s in specs], xs, ys, M=M)
+    bp.run()
+    torch.cuda.synchronize()
+    _status(bp)
+    for (s, rows, per_m, alpha), y in zip(checks, ys):
+        X, ref = per_m[M]
+        assert_parity(y.cpu().numpy().astype(np.float64)[:, rows], ref, X, alpha, f"{s.name} M={M}")
+    bp.close()
