@@ -18,9 +18,7 @@
 //    a row's code bytes (32 lanes x 32 B), residual-site bytes and
 //    {alpha, beta} words, completing on an mbarrier per ring slot.  While a
 //    CTA waits at the grid barrier its ring already fills with the next
-//    stage's rows; an L2 prefetch of its next tile, issued once its rows of
-//    the current group are consumed, keeps HBM busy through the combine, the
-//    barrier and the next prep.
+//    stage's rows, and the x of its next tile is warmed in L2.
 //  - Per group the CTA builds the fixed-point image of x: per 128-group g
 //    with largest exponent e_g, X_j = round(x_j * 2^(21 - e_g)), an integer
 //    below 2^22 in magnitude (exact when x_j is within 2^-14 of the group
@@ -495,9 +493,13 @@ __device__ __forceinline__ void build_image(const uint4 (&xr)[kMaxXChunks], int 
     }
 #pragma unroll
     for (int off = 8; off; off >>= 1) sum8 += __shfl_xor_sync(gmask, sum8, off);
-    const int gg = c >> 7, pos = c & 127, wl = (c >> 4) & 7, h = (c >> 3) & 1;
+    const int gg = c >> 7, pos = c & 127, h = (c >> 3) & 1;
     // limb image [group][word-in-group][limb][slot] (+4 words of padding per
-    // group): byte b of (word wl, limb L, slot q) = limb L of column 16 wl + 4 b + q
+    // group): byte b of (word wl, limb L, slot q) = limb L of column 16 wl + 4 b + q.
+    // A group read by a lane with bit 2 set is stored with its halves swapped
+    // (words 0-3 <-> 4-7), the order in which that lane holds its limbs, so
+    // that every lane reads its image front to back without bank conflicts.
+    const int wl = ((c >> 4) & 7) ^ ((gg & 4) ? 4 : 0);
     uint16_t* img16 = reinterpret_cast<uint16_t*>(limbs + (size_t)gg * kLimbStride);
 #pragma unroll
     for (int L2 = 0; L2 < 3; ++L2)
@@ -518,22 +520,6 @@ __device__ __forceinline__ void build_image(const uint4 (&xr)[kMaxXChunks], int 
     }
   }
   __syncthreads();
-}
-
-// Warm L2 with a tile (codes, sites, scales of its rows) and its x.
-__device__ __forceinline__ void prefetch_tile(const TileRec& t, const StreamItem& it) {
-  const int K = (int)t.G * kGroup;
-  const size_t G = t.G, n0 = (size_t)t.n0, n1 = (size_t)t.n0 + t.rows;
-  const size_t sb = it.k ? 4 : 2;
-  const size_t ranges[3][2] = {{n0 * (K / 4), n1 * (K / 4)}, {n0 * G * it.k, n1 * G * it.k}, {n0 * G * sb, n1 * G * sb}};
-  const unsigned char* base[3] = {reinterpret_cast<const unsigned char*>(it.codes), it.sites,
-                                  reinterpret_cast<const unsigned char*>(it.scales)};
-  for (int b = 0; b < 3; ++b) {
-    if (!base[b] || ranges[b][1] == ranges[b][0]) continue;
-    const size_t a = ranges[b][0] & ~(size_t)15, e = (ranges[b][1] + 15) & ~(size_t)15;
-    for (size_t o = a; o < e; o += 65536) prefetch_l2(base[b] + o, (uint32_t)min((size_t)65536, e - o));
-  }
-  prefetch_l2(it.x, (uint32_t)(K * 2));
 }
 
 __device__ __forceinline__ void prefetch_l1(const void* p) {
@@ -577,8 +563,9 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
   }
   build_image<SIGNED_TABLE>(xr, K, area, ap);
 
-  // the 96 limb words of this lane's group into registers; lanes with bit 2
-  // set swap the halves of their group (words 0-3 <-> 4-7), like their code reads
+  // the 96 limb words of this lane's group into registers; on lanes with bit
+  // 2 set register word w holds group word w ^ 4 (stored so in the image), as
+  // their code reads do
   const int col0 = W.s * kSliceCols + lane * kGroup;
   const bool active = worker && col0 < K;
   const int g = active ? col0 >> 7 : 0;
@@ -590,10 +577,9 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
     const uint32_t img = ptx::smem_u32(area + ap.limbs) + (uint32_t)g * kLimbStride * 4u;
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
-      const int wsw = hsw ? (w ^ 4) : w;
 #pragma unroll
       for (int L2 = 0; L2 < 3; ++L2) {
-        const uint4 v = lds128(img + (uint32_t)(wsw * 3 + L2) * 16u);
+        const uint4 v = lds128(img + (uint32_t)(w * 3 + L2) * 16u);
         lb[w][L2 * 4 + 0] = v.x; lb[w][L2 * 4 + 1] = v.y; lb[w][L2 * 4 + 2] = v.z; lb[w][L2 * 4 + 3] = v.w;
       }
     }
@@ -638,16 +624,15 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
     }
   }
 
-  // after its own rows, warm L2 with the CTA's next tile
-  if (tid == 0)
+  // the last warp (fewest rows) warms L2 with the x of the CTA's next tile
+  if (warp == (int)(blockDim.x / 32) - 1 && lane == 0)
     for (int jn = j + 1; jn < R.n_groups; ++jn) {
       const TileRec tn = R.sched[jn];
       if (tn.rows) {
-        prefetch_tile(tn, R.items[tn.item]);
+        prefetch_l2(R.items[tn.item].x, (uint32_t)tn.G * kGroup * 2u);
         break;
       }
     }
-
   const bool all_ok = !__syncthreads_or(!ok);
 
   // slices in order, WALB2 phase 2, one store per output
@@ -673,17 +658,18 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
 }
 
 // All CTAs of the launch meet here; `target` = CTAs x barriers passed so far.
+// Thread 0 arrives with a release add (the CTA barrier before it carries the
+// CTA's writes) and polls with acquire loads; the CTA barrier after it hands
+// the acquired view to every thread.
 __device__ __forceinline__ void grid_barrier(unsigned int* ctr, unsigned int target, int32_t* status) {
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(ctr, 1u);
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
     for (uint32_t it = 0; ld_acquire(ctr) < target; ++it)
       if (it >= kBarrierSpin) {
         if (status) atomicExch(status, (int32_t)WAL_ERR_TIMEOUT);
         break;
       }
-    __threadfence();
   }
   __syncthreads();
 }
