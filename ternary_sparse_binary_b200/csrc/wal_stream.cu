@@ -299,6 +299,7 @@ struct ProdState {
   int j, c, nc;
   uint32_t issued;    // chunks issued so far
   uint32_t consumed;  // chunks consumed so far
+  uint32_t slot;      // ring slot of the next chunk to issue (issued mod stages)
   WarpRing W;
 };
 __host__ __device__ inline uint32_t area_offset(int warps, int stages, int rpc) {
@@ -322,16 +323,20 @@ __device__ __forceinline__ void prod_seek(ProdState& ps, const TileRec* sched, i
   }
 }
 
-// Issue the producer's next chunk into ring slot st (if any is left).
-__device__ __forceinline__ void prod_issue(ProdState& ps, uint32_t ring, uint32_t mbar, uint32_t st,
+// Keep up to `stages` chunks in flight: issue the producer's next chunks (in
+// order, chunk n into slot n mod stages) while fewer are outstanding and, if
+// j_limit >= 0, while they belong to groups up to j_limit.
+__device__ __forceinline__ void prod_topup(ProdState& ps, uint32_t ring, uint32_t mbar, int stages,
                                            const TileRec* sched, int n_groups, const StreamItem* items, int warp,
-                                           const ChunkGeom& C) {
-  if (ps.j >= n_groups) return;
-  issue_chunk(ps.W, ring + st * C.bytes, mbar + st * 8u, ps.c, C);
-  ++ps.issued;
-  if (++ps.c == ps.nc) {
-    ++ps.j;
-    prod_seek(ps, sched, n_groups, items, warp, C.rpc);
+                                           const ChunkGeom& C, int j_limit) {
+  while (ps.j < n_groups && ps.issued - ps.consumed < (uint32_t)stages && (j_limit < 0 || ps.j <= j_limit)) {
+    issue_chunk(ps.W, ring + ps.slot * C.bytes, mbar + ps.slot * 8u, ps.c, C);
+    ++ps.issued;
+    if (++ps.slot == (uint32_t)stages) ps.slot = 0;
+    if (++ps.c == ps.nc) {
+      ++ps.j;
+      prod_seek(ps, sched, n_groups, items, warp, C.rpc);
+    }
   }
 }
 
@@ -431,7 +436,7 @@ __device__ __forceinline__ bool run_rows(const WarpRing& W, const RingCtx& R, ui
     __syncwarp();  // every lane has consumed the slot before it is refilled
     if (lane == 0) {
       ++R.ps->consumed;
-      prod_issue(*R.ps, R.ring, R.mbar, st, R.sched, R.n_groups, R.items, R.warp, C);
+      prod_topup(*R.ps, R.ring, R.mbar, R.stages, R.sched, R.n_groups, R.items, R.warp, C, -1);
     }
     if (++st == (uint32_t)R.stages) {
       st = 0;
@@ -624,6 +629,8 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
     }
   }
 
+  // keep this warp's ring full (a warp with no rows here has issued nothing since the first fill)
+  if (lane == 0) prod_topup(*R.ps, R.ring, R.mbar, R.stages, R.sched, R.n_groups, R.items, R.warp, R.C, -1);
   // the last warp (fewest rows) warms L2 with the x of the CTA's next tile
   if (warp == (int)(blockDim.x / 32) - 1 && lane == 0)
     for (int jn = j + 1; jn < R.n_groups; ++jn) {
@@ -714,9 +721,13 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
     R.ps->j = 0;
     R.ps->issued = 0;
     R.ps->consumed = 0;
+    R.ps->slot = 0;
     prod_seek(*R.ps, sched, n_groups, items, warp, R.C.rpc);
-    for (int s0 = 0; s0 < stages; ++s0)
-      prod_issue(*R.ps, R.ring, R.mbar, (uint32_t)s0, sched, n_groups, items, warp, R.C);
+    // the first fill stays inside the CTA's first group with rows; the
+    // run-ahead into later groups starts once that group is under way
+    int j0 = 0;
+    while (j0 + 1 < n_groups && sched[j0].rows == 0) ++j0;
+    prod_topup(*R.ps, R.ring, R.mbar, stages, sched, n_groups, items, warp, R.C, j0);
   }
   __syncwarp();
 
