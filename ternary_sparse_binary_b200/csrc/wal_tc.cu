@@ -40,6 +40,9 @@
 //             residual plane is zeroed and the k sites scattered as +-beta.
 //             Then the same warps run the epilogue:
 //             y[m][n] = (D + D2 2^t_m) 2^-sc_m.
+// With few row tiles the K range is split over CTAs (ks splits of whole
+// 128-column groups); each split writes its raw sums and a third launch adds
+// the splits in order and applies 2^-sc_m.  The WALB2 MMA belongs to split 0.
 // All mbarrier waits are bounded; one that gives up records WAL_ERR_TIMEOUT in
 // the status word and its role stops issuing work.
 #include "wal_internal.h"
@@ -85,6 +88,8 @@ struct TcParams {
   const float2* scal;
   float* Y;
   int ldy, N, K, r, M, M_tile, stages, n_tiles_n;
+  int ks, gps;         // K splits and 128-column groups per split
+  float* part;         // ks > 1: raw partial sums [ks][M][N]
   uint32_t d2_col;     // tensor-memory column of D2
   uint32_t tmem_cols;  // allocated tensor-memory columns
   int32_t* status;
@@ -134,6 +139,13 @@ __global__ void __launch_bounds__(kPrepThreads) tc_prep_kernel(const TcPrepParam
   const int sc = mx ? 14 - ilog2f_bits(mx << 16) : 0;
   const double f = pow2d(sc);
 
+  // the V bit planes in shared memory (coalesced), read per 16 columns below
+  extern __shared__ __align__(16) uint32_t s_v[];  // [r][K/32]
+  const int vwords = p.r * (p.K / 32);
+  for (int i = tid; i < vwords / 4; i += kPrepThreads)
+    reinterpret_cast<uint4*>(s_v)[i] = __ldg(reinterpret_cast<const uint4*>(p.vbits) + i);
+  __syncthreads();
+
   float acc[WAL_MAX_RANK];
 #pragma unroll
   for (int q = 0; q < WAL_MAX_RANK; ++q) acc[q] = 0.f;
@@ -168,7 +180,7 @@ __global__ void __launch_bounds__(kPrepThreads) tc_prep_kernel(const TcPrepParam
 #pragma unroll
       for (int q = 0; q < WAL_MAX_RANK; ++q) {
         if (q < p.r) {
-          const uint32_t bits = (__ldg(p.vbits + (size_t)q * (p.K / 32) + (b >> 1)) >> (16 * (b & 1))) & 0xFFFFu;
+          const uint32_t bits = (s_v[q * (p.K / 32) + (b >> 1)] >> (16 * (b & 1))) & 0xFFFFu;
           float s = 0.f;
 #pragma unroll
           for (int j = 0; j < 16; ++j) s += __uint_as_float(__float_as_uint(xs[j]) ^ (((bits >> j) & 1u) << 31));
@@ -287,10 +299,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
   auto a_r = [&](int s) { return base + (uint32_t)s * stage_bytes + kATile; };
   auto b_t = [&](int s) { return base + (uint32_t)s * stage_bytes + kATile * (kHasR ? 2u : 1u); };
 
-  const int n_tile = blockIdx.x % p.n_tiles_n, mt = blockIdx.x / p.n_tiles_n;
-  const int G = p.K / 128, KB = p.K / kBlockK;
-  const bool has_lr = p.r > 0;
-  const int n_iter = KB + (has_lr ? 1 : 0);
+  // CTA -> (row tile, K split, activation tile); row tiles vary fastest so
+  // that concurrent CTAs share B tiles in L2
+  const int n_tile = blockIdx.x % p.n_tiles_n;
+  const int split = (blockIdx.x / p.n_tiles_n) % p.ks, mt = blockIdx.x / (p.n_tiles_n * p.ks);
+  const int KB = p.K / kBlockK;
+  const int g0 = split * p.gps, G = min(p.K / 128, g0 + p.gps);  // this split's groups [g0, G)
+  const int KBl = 2 * (G - g0), kb0 = 2 * g0;                     // its K-blocks [kb0, kb0 + KBl)
+  const bool has_lr = p.r > 0 && split == 0;                       // the WALB2 MMA belongs to split 0
+  const int n_iter = KBl + (has_lr ? 1 : 0);
   const uint32_t ncols = p.tmem_cols;
 
   if (tid == 0) {
@@ -318,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
         const int s = i % S;
         const uint32_t ph = (uint32_t)(i / S) & 1u;
         if (!mbar_wait(empty(s), ph ^ 1u, p.status)) break;
-        const char* src = i < KB ? p.xt + ((size_t)mt * KB + i) * b_bytes : p.zt + (size_t)mt * b_bytes;
+        const char* src = i < KBl ? p.xt + ((size_t)mt * KB + kb0 + i) * b_bytes : p.zt + (size_t)mt * b_bytes;
         mbar_arrive_expect_tx(b_full(s), b_bytes);
         bulk_g2s(b_t(s), src, b_bytes, b_full(s));
       }
@@ -328,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(kRows, (uint32_t)p.M_tile);
       bool ok = true;
-      for (int i = 0; i < KB && ok; ++i) {
+      for (int i = 0; i < KBl && ok; ++i) {
         const int s = i % S;
         const uint32_t ph = (uint32_t)(i / S) & 1u;
         ok = mbar_wait(b_full(s), ph, p.status) && mbar_wait(a_full(s), ph, p.status);
@@ -343,8 +360,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
         mma_commit(empty(s));
       }
       if (ok && has_lr) {
-        const int s = KB % S;
-        const uint32_t ph = (uint32_t)(KB / S) & 1u;
+        const int s = KBl % S;
+        const uint32_t ph = (uint32_t)(KBl / S) & 1u;
         ok = mbar_wait(b_full(s), ph, p.status) && mbar_wait(a_full(s), ph, p.status);
         if (ok) {
           tc_fence_after();
@@ -367,13 +384,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
     const uint32_t r7 = (uint32_t)row & 7u;
     bool ok = true;
 
+    const int GK = p.K / 128;
     GroupLoad<KS> cur = {}, nxt = {};
-    if (live) cur = load_group<KS>(p, n, 0, h, G);
-    if (live && G > 1) nxt = load_group<KS>(p, n, 1, h, G);
-    for (int g = 0; g < G && ok; ++g) {
+    if (live) cur = load_group<KS>(p, n, g0, h, GK);
+    if (live && g0 + 1 < G) nxt = load_group<KS>(p, n, g0 + 1, h, GK);
+    for (int g = g0; g < G && ok; ++g) {
       GroupLoad<KS> nn = {};
-      if (live && g + 2 < G) nn = load_group<KS>(p, n, g + 2, h, G);
-      const int i = 2 * g + h, s = i % S;
+      if (live && g + 2 < G) nn = load_group<KS>(p, n, g + 2, h, GK);
+      const int i = 2 * (g - g0) + h, s = i % S;
       const uint32_t ph = (uint32_t)(i / S) & 1u;
       ok = mbar_wait(empty(s), ph ^ 1u, p.status);
       if (!ok) break;
@@ -411,9 +429,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
       nxt = nn;
     }
     // WALB2 phase-2 operand A_lr[n] = (+-s_0 .. +-s_{r-1}, +-s_0 .. +-s_{r-1}, 0 ...)
-    if (ok && has_lr && h == (KB & 1)) {
-      const int s = KB % S;
-      const uint32_t ph = (uint32_t)(KB / S) & 1u;
+    if (ok && has_lr && h == (KBl & 1)) {
+      const int s = KBl % S;
+      const uint32_t ph = (uint32_t)(KBl / S) & 1u;
       ok = mbar_wait(empty(s), ph ^ 1u, p.status);
       if (ok) {
         const uint32_t u = live ? __ldg(p.ubits + (size_t)n * ((p.r + 31) / 32)) : 0u;
@@ -462,8 +480,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
           const uint2 sv = lds64(scal_s + 8u * col);
           float y = __uint_as_float(d[j]);
           if (has_lr) y = fmaf(__uint_as_float(e[j]), __uint_as_float(sv.y), y);
-          y *= __uint_as_float(sv.x);
-          if (live && m < p.M) p.Y[(size_t)m * p.ldy + n] = y;
+          if (p.ks == 1) {
+            y *= __uint_as_float(sv.x);
+            if (live && m < p.M) p.Y[(size_t)m * p.ldy + n] = y;
+          } else if (live && m < p.M) {
+            p.part[((size_t)split * p.M + m) * p.N + n] = y;  // raw: scaled by 2^-sc_m after the sum
+          }
         }
       }
     }
@@ -473,6 +495,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, ncols);
+  }
+}
+
+// Split-K: y[m][n] = 2^-sc_m * sum over splits (in order) of the raw partials.
+__global__ void __launch_bounds__(256) tc_reduce_kernel(const float* __restrict__ part, const float2* __restrict__ scal,
+                                                        float* Y, int ldy, int M, int N, int ks) {
+  const size_t total = (size_t)M * N;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int m = (int)(i / N), n = (int)(i % N);
+    float acc = 0.f;
+    for (int s2 = 0; s2 < ks; ++s2) acc += __ldg(part + (size_t)s2 * total + i);
+    Y[(size_t)m * ldy + n] = acc * __ldg(&scal[m].x);
   }
 }
 
@@ -488,6 +522,7 @@ int tc_init() {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&g_tc_smem_limit, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_tc_smem_limit);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_tc_smem_limit);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_tc_smem_limit);
@@ -522,10 +557,34 @@ int plan_tc(const wal_matrix* m, int M, TcPlan* out) {
   P.smem = extra + (uint32_t)P.stages * stage_bytes;
   const uint32_t d2 = pow2_ceil((uint32_t)P.M_tile);
   P.tmem_cols = std::max(32u, d2 * (m->r > 0 ? 2u : 1u));
+  // K splits: with few row tiles, split K so the grid fills the SMs.  Cost
+  // model in microseconds: waves x (K-blocks per split + about 4 of fixed
+  // work) x about 1 us per K-block, plus the split sums' traffic (ks partial
+  // planes read, one written) at about 3 TB/s.  The B200's 148 SMs are a
+  // constant here so the plan (and the workspace size) do not depend on
+  // device queries.
+  const int G = m->K / 128, tiles = P.n_tiles_n * P.n_mt;
+  constexpr int kPlanSms = 148;
+  double best = 1e30;
+  P.ks = 1;
+  P.gps = G;
+  for (int ks = 1; ks <= std::min(G, 16); ++ks) {
+    const int gps = (G + ks - 1) / ks, eff = (G + gps - 1) / gps;
+    if (eff != ks) continue;
+    const int waves = (tiles * ks + kPlanSms - 1) / kPlanSms;
+    const double reduce_us = ks > 1 ? (double)(ks + 1) * M * m->N * 4.0 / 3.0e6 : 0.0;
+    const double est = (double)waves * (2.0 * gps + 4.0) + reduce_us;
+    if (est < best - 1e-9) {
+      best = est;
+      P.ks = ks;
+      P.gps = gps;
+    }
+  }
   P.off_scal = 0;
   P.off_zt = align_up(256 + (size_t)P.M_pad * 8, 1024);
   P.off_xt = align_up(P.off_zt + (m->r > 0 ? (size_t)P.n_mt * b_bytes : 0), 1024);
-  P.total = P.off_xt + (size_t)P.M_pad * m->K * 2;
+  P.off_part = align_up(P.off_xt + (size_t)P.M_pad * m->K * 2, 1024);
+  P.total = P.off_part + (P.ks > 1 ? (size_t)P.ks * M * m->N * 4 : 0);
   *out = P;
   return WAL_OK;
 }
@@ -552,7 +611,8 @@ int launch_tc(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, 
   pp.zt = data + P.off_zt;
   pp.scal = reinterpret_cast<float2*>(data + P.off_scal);
   pp.status = status;
-  tc_prep_kernel<<<P.M_pad, kPrepThreads, 0, stream>>>(pp);
+  const size_t vbytes = (size_t)m->r * (m->K / 8);  // <= 32 * 24576 / 8 = 96 KB
+  tc_prep_kernel<<<P.M_pad, kPrepThreads, vbytes, stream>>>(pp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("tc_prep_kernel launch: ") + cudaGetErrorString(e));
 
@@ -561,10 +621,12 @@ int launch_tc(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, 
   tp.xt = pp.xt; tp.zt = pp.zt; tp.scal = pp.scal;
   tp.Y = Y; tp.ldy = ldy; tp.N = m->N; tp.K = m->K; tp.r = m->r; tp.M = M; tp.M_tile = P.M_tile;
   tp.stages = P.stages; tp.n_tiles_n = P.n_tiles_n;
+  tp.ks = P.ks; tp.gps = P.gps;
+  tp.part = reinterpret_cast<float*>(data + P.off_part);
   tp.d2_col = m->r > 0 ? P.tmem_cols / 2 : P.tmem_cols;
   tp.tmem_cols = P.tmem_cols;
   tp.status = status;
-  const dim3 grid(P.n_tiles_n * P.n_mt);
+  const dim3 grid(P.n_tiles_n * P.ks * P.n_mt);
   switch (m->k) {
     case 0: tc_kernel<0><<<grid, kThreads, P.smem, stream>>>(tp); break;
     case 2: tc_kernel<2><<<grid, kThreads, P.smem, stream>>>(tp); break;
@@ -573,6 +635,13 @@ int launch_tc(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, 
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("tc_kernel launch: ") + cudaGetErrorString(e));
+  if (P.ks > 1) {
+    const size_t total = (size_t)M * m->N;
+    const int blocks = (int)std::min<size_t>((total + 255) / 256, 148 * 8);
+    tc_reduce_kernel<<<blocks, 256, 0, stream>>>(tp.part, tp.scal, Y, ldy, M, m->N, P.ks);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("tc_reduce_kernel launch: ") + cudaGetErrorString(e));
+  }
   return WAL_OK;
 }
 

@@ -17,10 +17,11 @@ struct TcPlan {
   int M_tile;     // activation rows per tile (MMA N), multiple of 16, <= 256
   int M_pad;      // n_mt * M_tile
   int stages;     // pipeline depth
+  int ks, gps;    // K splits and 128-column groups per split
   uint32_t smem;  // dynamic shared memory per CTA
   uint32_t tmem_cols;
   // workspace offsets from the 256-byte aligned base
-  size_t off_scal, off_zt, off_xt, total;
+  size_t off_scal, off_zt, off_xt, off_part, total;
 };
 
 int plan_tc(const wal_matrix* m, int M, TcPlan* out);
