@@ -21,6 +21,7 @@ from .gen import (  # noqa: F401
     body_plan,
     config_plan,
     gen_matrix,
+    gen_pq2,
     workload_id,
     WORKLOAD_IDS,
     CONFIG_SEED,

@@ -193,7 +193,7 @@ def body_plan(layers, layer_roles, k_by_role, r_default, config_id, n_lowrank=No
 
 
 # workload name -> seed id used in every SeedSequence of that workload
-WORKLOAD_IDS = {"single": 0, "layer8b": 1, "body8b": 2, "body27b": 3, "sweep": 4}
+WORKLOAD_IDS = {"single": 0, "layer8b": 1, "body8b": 2, "body27b": 3, "sweep": 4, "pq2_body8b": 5}
 
 
 def config_plan(workload):
@@ -205,6 +205,8 @@ def config_plan(workload):
     body27b: 64 layers x 7 = 448 27B-shaped matrices; k by role (MLP 8, q/k/v 4,
              o 2), a seeded 45 (10 %) forced to k=0, a seeded 152 carry r=8.
     sweep  : gate 4096->12288 and down 12288->4096, k=8, r=16 (batch sweep).
+    pq2_body8b: the 252 matrices of body8b as plain ternary (k=0, r=0), the
+             PQ2_0 block format's workload.
     """
     wid = WORKLOAD_IDS[workload] if isinstance(workload, str) else int(workload)
     if wid == 0:
@@ -218,6 +220,8 @@ def config_plan(workload):
     if wid == 4:
         return [MatrixSpec("gate", 12288, 4096, 8, 16, 0, 0, 0),
                 MatrixSpec("down", 4096, 12288, 8, 16, 1, 1, 0)]
+    if wid == 5:
+        return body_plan(36, LAYER_8B, 0, 0, wid)
     raise ValueError(f"unknown workload {workload}")
 
 
@@ -228,3 +232,11 @@ def workload_id(workload) -> int:
 def gen_matrix(workload, spec: MatrixSpec) -> Components:
     """Components of one matrix of a workload, seeded by (workload, matrix index)."""
     return gen_components(spec.N, spec.K, spec.k, spec.r, workload_id(workload), spec.index)
+
+
+def gen_pq2(N: int, K: int, config_id: int = 0, matrix_index: int = 0):
+    """One plain-ternary matrix for the PQ2_0 block format: T iid as in
+    gen_components and one scale d = fp16(|N(0, 0.02)|) per (row, 128-group).
+    Returns (T int8 [N, K], d uint16 fp16 bits [N, K/128])."""
+    c = gen_components(N, K, 0, 0, config_id, matrix_index)
+    return c.T, c.alpha
