@@ -4,6 +4,8 @@
 Default run (one GPU):  python bench.py
 Replicas on N GPUs:     python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N
 Oracle (CPU) arm:       python bench.py --impl reference
+Second workload:        python bench.py --workload pq2_body8b   (the same 252 shapes as
+                        plain-ternary PQ2_0 blocks, 34 bytes per 128 weights)
 
 Prints ONE JSON line (rank 0).  The metric is microseconds per body pass at
 batch 1 (lower is better) together with the weight stream in GB/s against the
@@ -37,7 +39,32 @@ def parse():
     ap.add_argument("--impl", choices=["wal", "reference"], default="wal")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-matrices", type=int, default=4)
-    return ap.parse_args()
+    ap.add_argument("--workload", choices=["body8b", "pq2_body8b"], default="body8b")
+    a = ap.parse_args()
+    global WORKLOAD
+    WORKLOAD = a.workload
+    return a
+
+
+def is_pq2():
+    return WORKLOAD == "pq2_body8b"
+
+
+def workload_text():
+    if is_pq2():
+        return ("8B-shaped body pass in PQ2_0: 36 layers x 7 plain-ternary matrices (q,k,v,o 4096-wide; gate/up "
+                "4096->12288; down 12288->4096), 34-byte blocks (FP16 scale + 32 code bytes) per 128 weights, "
+                "batch 1, one CUDA graph holding one persistent cooperative launch, 144 dependency stages "
+                "separated by grid barriers")
+    return ("8B-shaped body pass: 36 layers x 7 matrices (q,k,v,o 4096-wide; gate/up 4096->12288; "
+            "down 12288->4096), k=8 sites per 128-group, 213 of 252 with WALB2 r=8, batch 1, "
+            "one CUDA graph holding one persistent cooperative launch, 144 dependency stages "
+            "separated by grid barriers")
+
+
+def seed_id():
+    from wal_synth import workload_id
+    return workload_id(WORKLOAD)
 
 
 def dist_env():
@@ -109,9 +136,19 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # workload
 # ---------------------------------------------------------------------------
+def weight_bytes(s):
+    """Algorithmic (payload) bytes of one matrix, before the 16-byte padding.
+    Layout v1: codes N K / 4, sites N G k, scales N G (4 | 2), U N ceil(r/32) 4,
+    V r K / 8, per-rank scales 2 r.  PQ2_0: 34 bytes per 128 weights."""
+    G = s.K // 128
+    if is_pq2():
+        return s.N * G * 34
+    return (s.N * s.K // 4 + s.N * G * s.k + s.N * G * (4 if s.k else 2) + s.N * ((s.r + 31) // 32) * 4
+            + s.r * s.K // 8 + 2 * s.r)
+
+
 def algorithmic_bytes(specs):
-    import oracle  # sizes only: payload bytes of layout v1
-    wbytes = sum(sum(oracle.payload_sizes(s.N, s.K, s.k, s.r)) for s in specs)
+    wbytes = sum(weight_bytes(s) for s in specs)
     io = sum(2 * s.K + 4 * s.N for s in specs)
     return wbytes, io
 
@@ -119,20 +156,25 @@ def algorithmic_bytes(specs):
 def build_workload(device):
     import torch
     import ternary_sparse_binary_b200 as wal
-    from wal_synth import config_plan, gen_matrix, gen_x
+    from wal_synth import config_plan, gen_matrix, gen_pq2, gen_x
     specs = config_plan(WORKLOAD)
     mats = []
     t0 = time.time()
     for s in specs:
-        c = gen_matrix(WORKLOAD, s)
-        mats.append(wal.PackedMatrix(wal.pack_host(c), s.N, s.K, s.k, s.r, device=device))
-        del c
+        if is_pq2():
+            T, d = gen_pq2(s.N, s.K, seed_id(), s.index)
+            mats.append(wal.Pq2Matrix(wal.pack_pq2_host(T, d, s.N, s.K), s.N, s.K, device=device))
+            del T, d
+        else:
+            c = gen_matrix(WORKLOAD, s)
+            mats.append(wal.PackedMatrix(wal.pack_host(c), s.N, s.K, s.k, s.r, device=device))
+            del c
     setup_s = time.time() - t0
     xoff, yoff = [0], [0]
     for s in specs:
         xoff.append(xoff[-1] + s.K)
         yoff.append(yoff[-1] + s.N)
-    x_host = np.concatenate([gen_x(s.K, 1, 2, s.index)[0] for s in specs]).view(np.int16)
+    x_host = np.concatenate([gen_x(s.K, 1, seed_id(), s.index)[0] for s in specs]).view(np.int16)
     x_pinned = torch.from_numpy(x_host).pin_memory()
     x_dev = x_pinned.to(device)
     y_dev = torch.empty(yoff[-1], dtype=torch.float32, device=device)
@@ -155,9 +197,9 @@ def time_gate_product(w, device, reps=20):
     the first gate matrix, L2 flushed between launches."""
     import torch
     import ternary_sparse_binary_b200 as wal
-    import oracle
     idx = next(i for i, s in enumerate(w["specs"]) if s.name.endswith("gate"))
     s, pm = w["specs"][idx], w["mats"][idx]
+    pq2 = is_pq2()
     x = w["x_dev"][: s.K]
     y = torch.empty(s.N, dtype=torch.float32, device=device)
     nb = pm.workspace_bytes(1)
@@ -170,20 +212,26 @@ def time_gate_product(w, device, reps=20):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        wal.wal_gemv(pm.desc, x.data_ptr(), y.data_ptr(), ws.data_ptr(), nb, stream.cuda_stream)
+        if pq2:
+            wal.wal_pq2_gemm(pm.desc, x.data_ptr(), 1, s.K, y.data_ptr(), s.N, ws.data_ptr(), nb, stream.cuda_stream)
+        else:
+            wal.wal_gemv(pm.desc, x.data_ptr(), y.data_ptr(), ws.data_ptr(), nb, stream.cuda_stream)
         e1.record(stream)
         e1.synchronize()
         if i >= 3:
             durs.append(e0.elapsed_time(e1) * 1e-3)
-    wbytes = sum(oracle.payload_sizes(s.N, s.K, s.k, s.r)) + 2 * s.K + 4 * s.N
+    wbytes = weight_bytes(s) + 2 * s.K + 4 * s.N
     dur = float(np.mean(durs))
-    return {"matrix": f"{s.name} {s.K}->{s.N} k={s.k} r={s.r}", "bytes_per_launch": wbytes,
+    what = f"{s.name} {s.K}->{s.N} PQ2_0" if pq2 else f"{s.name} {s.K}->{s.N} k={s.k} r={s.r}"
+    return {"matrix": what, "bytes_per_launch": wbytes,
             "us_per_launch": dur * 1e6, "gbs": wbytes / dur / 1e9}
 
 
 def load_traffic(kernel="stream_kernel"):
     """Traffic per launch from the committed ncu summary, if it was taken on
-    the current kernel source."""
+    the current kernel source (and the workload's format)."""
+    if is_pq2():
+        kernel = "stream_kernel_pq2"
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
@@ -203,7 +251,8 @@ def cpu_baseline(specs, n_sample):
     n_sample matrices (one of each role, cycling), scaled to a full pass by
     weight count."""
     import oracle
-    from wal_synth import gen_matrix, gen_x
+    from oracle import pq2_oracle
+    from wal_synth import gen_matrix, gen_pq2, gen_x
     try:
         from threadpoolctl import threadpool_info
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
@@ -219,10 +268,16 @@ def cpu_baseline(specs, n_sample):
             break
     t_total, w_sample = 0.0, 0
     for s in sample:
-        c = gen_matrix(WORKLOAD, s)
-        x = gen_x(s.K, 1, 2, s.index)[0]
-        t0 = time.perf_counter()
-        oracle.matvec(c, x)
+        x = gen_x(s.K, 1, seed_id(), s.index)[0]
+        if is_pq2():
+            T, d = gen_pq2(s.N, s.K, seed_id(), s.index)
+            buf = pq2_oracle.pack(pq2_oracle.Pq2(s.N, s.K, T, d))
+            t0 = time.perf_counter()
+            pq2_oracle.matmul(pq2_oracle.unpack(buf, s.N, s.K), x.reshape(1, -1))
+        else:
+            c = gen_matrix(WORKLOAD, s)
+            t0 = time.perf_counter()
+            oracle.matvec(c, x)
         t_total += time.perf_counter() - t0
         w_sample += s.N * s.K
     w_all = sum(s.N * s.K for s in specs)
@@ -252,7 +307,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1e3, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "8B-shaped body pass: 36 layers x 7 matrices, k=8, 213 with WALB2 r=8, batch 1"},
+            "config": {"workload": workload_text()},
             "cpu_baseline": cb,
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -345,12 +400,9 @@ def run_wal(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "int32+f32 (dp4a on a 24-bit fixed-point x image, FP32 scales and accumulation)",
             "data": "synthetic",
-            "config": {"workload": "8B-shaped body pass: 36 layers x 7 matrices (q,k,v,o 4096-wide; gate/up 4096->12288; "
-                                   "down 12288->4096), k=8 sites per 128-group, 213 of 252 with WALB2 r=8, batch 1, "
-                                   "one CUDA graph holding one persistent cooperative launch, 144 dependency stages "
-                                   "separated by grid barriers",
+            "config": {"workload": workload_text(),
                        "weights_bytes": wbytes, "io_bytes": iobytes,
-                       "l2": "inputs larger than L2 (2.39 GB of packed weights per pass vs 126 MB L2)",
+                       "l2": f"inputs larger than L2 ({wbytes / 1e9:.2f} GB of packed weights per pass vs 126 MB L2)",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "step_us_p10_p50_p90": [float(np.percentile(per_step, q)) for q in (10, 50, 90)],
                        "weight_gbs": gbs, "setup_s": round(w["setup_s"], 1)},

@@ -175,6 +175,51 @@ int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n_mats,
                   void* ws, size_t ws_bytes, wal_stream_t stream);
 void wal_body_plan_destroy(wal_body_plan* plan);
 
+/* ---- PQ2_0: the plain-ternary block format ---------------------------------
+ * The WAL2-Ternary-27B card (section on bit widths) describes PQ2_0, the
+ * format of its fast native GGUF: 32 bytes of 2-bit codes plus a 2-byte FP16
+ * scale for every 128 weights (34 bytes, 2.125 bits per weight), three of
+ * the four codes in use.  W[n][128 g + j] = d[n][g] * T[n][128 g + j]: the
+ * direct-packed product with k = 0 and r = 0, scale and codes side by side.
+ * This library's reading of the block (the card does not give the order):
+ *   block (n, g) at byte 34 * (n * G + g): uint16 fp16 bits d (little
+ *   endian), then 32 code bytes, trit j of the block in code byte j / 4 at
+ *   bits 2 * (j % 4), code c = t + 1 (3 reserved), as in layout v1.
+ *   The buffer is zero-padded to a multiple of 16 bytes (wal_pq2_bytes).
+ * The product streams it with its own specialisation of the decode-GEMV (no
+ * site table, no low-rank term); decode errors are not checked at run time. */
+typedef struct wal_pq2_matrix {
+  int32_t N, K;              /* K a positive multiple of 128, at most 24576 */
+  const uint8_t* blocks;     /* device pointer, 16-byte aligned */
+} wal_pq2_matrix;
+
+/* Bytes of a PQ2_0 buffer for an N x K matrix (34 * N * K / 128 rounded up
+ * to 16); 0 on a bad shape.  Host only. */
+size_t wal_pq2_bytes(int N, int K);
+
+/* Pack T [N][K] int8 in {-1,0,1} and d [N][K/128] fp16 bits into the PQ2_0
+ * buffer `out` (host memory, wal_pq2_bytes(N, K) bytes, padding zeroed).
+ * Host only, multi-threaded.  WAL_ERR_FORMAT when T leaves {-1,0,1}. */
+int wal_pq2_pack(const int8_t* T, const uint16_t* d, int N, int K, void* out);
+
+/* Scratch bytes of wal_pq2_gemm (1 <= M <= 16); 0 on a bad argument. */
+size_t wal_pq2_workspace_bytes(const wal_pq2_matrix* m, int M);
+
+/* Y[M][ldy] = X[M][ldx] W^T for a PQ2_0 matrix, 1 <= M <= 16 (one product
+ * per activation row in one launch; the batch-1 decode-GEMV).  X bf16 bits,
+ * 16-byte aligned, ldx >= K and a multiple of 8; Y fp32, ldy >= N.
+ * Asynchronous; a bounded wait that gives up records WAL_ERR_TIMEOUT in the
+ * workspace header (wal_device_status). */
+int wal_pq2_gemm(const wal_pq2_matrix* m, const uint16_t* X, int M, int ldx, float* Y, int ldy, void* ws,
+                 size_t ws_bytes, wal_stream_t stream);
+
+/* Body pass over PQ2_0 matrices: the same contract as wal_body_pass (stages,
+ * plan, graph replay, workspace ownership), with every matrix in PQ2_0. */
+size_t wal_pq2_body_workspace_bytes(const wal_pq2_matrix* mats, int n_mats, int M);
+int wal_pq2_body_pass(wal_body_plan** plan, const wal_pq2_matrix* mats, int n_mats, const int32_t* stage_of,
+                      const uint16_t* const* xs, float* const* ys, int M, void* ws, size_t ws_bytes,
+                      wal_stream_t stream);
+
 const char* wal_status_string(int status);
 const char* wal_last_error(void);
 

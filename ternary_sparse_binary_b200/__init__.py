@@ -12,5 +12,7 @@ from ._abi import (  # noqa: F401
     wal_packed_sizes, wal_pack_matrix, wal_validate, wal_unpack_matrix, wal_workspace_bytes,
     wal_gemv, wal_gemm_small_m, wal_gemm_tc_noalloc, wal_device_status, wal_body_workspace_bytes, wal_body_pass,
     wal_body_plan_destroy, wal_status_string, wal_last_error,
+    wal_pq2_matrix, wal_pq2_bytes, wal_pq2_pack, wal_pq2_workspace_bytes, wal_pq2_gemm,
+    wal_pq2_body_workspace_bytes, wal_pq2_body_pass,
 )
-from .packed import PackedMatrix, pack_host, to_device, BodyPass  # noqa: F401
+from .packed import PackedMatrix, Pq2Matrix, pack_host, pack_pq2_host, to_device, BodyPass  # noqa: F401

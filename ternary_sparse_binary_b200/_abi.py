@@ -25,6 +25,8 @@ EXPORTED_SYMBOLS = [
     "wal_packed_sizes", "wal_pack_matrix", "wal_validate", "wal_unpack_matrix",
     "wal_workspace_bytes", "wal_gemv", "wal_gemm_small_m", "wal_gemm_tc_noalloc", "wal_device_status",
     "wal_body_workspace_bytes", "wal_body_pass", "wal_body_plan_destroy",
+    "wal_pq2_bytes", "wal_pq2_pack", "wal_pq2_workspace_bytes", "wal_pq2_gemm",
+    "wal_pq2_body_workspace_bytes", "wal_pq2_body_pass",
     "wal_status_string", "wal_last_error",
 ]
 
@@ -41,6 +43,10 @@ class wal_matrix(ctypes.Structure):
         ("codes", ctypes.c_void_p), ("sites", ctypes.c_void_p), ("scales", ctypes.c_void_p),
         ("u_bits", ctypes.c_void_p), ("v_bits", ctypes.c_void_p), ("lr_scale", ctypes.c_void_p),
     ]
+
+
+class wal_pq2_matrix(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("blocks", ctypes.c_void_p)]
 
 
 def _load():
@@ -70,6 +76,17 @@ lib.wal_body_pass.argtypes = [ctypes.POINTER(_vp), _MP, _i, ctypes.POINTER(ctype
                               ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp, _sz, _vp]
 lib.wal_body_plan_destroy.argtypes = [_vp]
 lib.wal_body_plan_destroy.restype = None
+_PP = ctypes.POINTER(wal_pq2_matrix)
+lib.wal_pq2_bytes.argtypes = [_i, _i]
+lib.wal_pq2_bytes.restype = _sz
+lib.wal_pq2_pack.argtypes = [_vp, _vp, _i, _i, _vp]
+lib.wal_pq2_workspace_bytes.argtypes = [_PP, _i]
+lib.wal_pq2_workspace_bytes.restype = _sz
+lib.wal_pq2_gemm.argtypes = [_PP, _vp, _i, _i, _vp, _i, _vp, _sz, _vp]
+lib.wal_pq2_body_workspace_bytes.argtypes = [_PP, _i, _i]
+lib.wal_pq2_body_workspace_bytes.restype = _sz
+lib.wal_pq2_body_pass.argtypes = [ctypes.POINTER(_vp), _PP, _i, ctypes.POINTER(ctypes.c_int32),
+                                  ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp, _sz, _vp]
 lib.wal_status_string.argtypes = [_i]
 lib.wal_status_string.restype = ctypes.c_char_p
 lib.wal_last_error.argtypes = []
@@ -150,3 +167,35 @@ def wal_body_pass(plan, mats, stage_of, xs, ys, M, ws, ws_bytes, stream):
 
 def wal_body_plan_destroy(plan):
     lib.wal_body_plan_destroy(plan)
+
+
+def wal_pq2_bytes(N, K):
+    return int(lib.wal_pq2_bytes(N, K))
+
+
+def wal_pq2_pack(T, d, N, K, out):
+    return _check(lib.wal_pq2_pack(T, d, N, K, out), "wal_pq2_pack")
+
+
+def wal_pq2_workspace_bytes(m, M):
+    return int(lib.wal_pq2_workspace_bytes(ctypes.byref(m), M))
+
+
+def wal_pq2_gemm(m, X, M, ldx, Y, ldy, ws, ws_bytes, stream):
+    return _check(lib.wal_pq2_gemm(ctypes.byref(m), X, M, ldx, Y, ldy, ws, ws_bytes, stream), "wal_pq2_gemm")
+
+
+def wal_pq2_body_workspace_bytes(mats, M):
+    arr = (wal_pq2_matrix * len(mats))(*mats)
+    return int(lib.wal_pq2_body_workspace_bytes(arr, len(mats), M))
+
+
+def wal_pq2_body_pass(plan, mats, stage_of, xs, ys, M, ws, ws_bytes, stream):
+    """plan: a ctypes.c_void_p holding the plan handle (None on the first call)."""
+    n = len(mats)
+    marr = (wal_pq2_matrix * n)(*mats)
+    sarr = (ctypes.c_int32 * n)(*stage_of)
+    xarr = (_vp * n)(*xs)
+    yarr = (_vp * n)(*ys)
+    return _check(lib.wal_pq2_body_pass(ctypes.byref(plan), marr, n, sarr, xarr, yarr, M, ws, ws_bytes,
+                                        stream), "wal_pq2_body_pass")

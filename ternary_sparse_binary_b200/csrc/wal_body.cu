@@ -20,6 +20,7 @@ StreamItem make_item(const wal_matrix* m, const uint16_t* x, float* y);
 using namespace wal;
 
 struct wal_body_plan {
+  int fmt = kFmtV1;
   std::vector<wal_matrix> mats;
   std::vector<int32_t> stages;
   std::vector<const uint16_t*> xs;
@@ -39,9 +40,10 @@ bool same_matrix(const wal_matrix& a, const wal_matrix& b) {
          a.scales == b.scales && a.u_bits == b.u_bits && a.v_bits == b.v_bits && a.lr_scale == b.lr_scale;
 }
 
-bool plan_matches(const wal_body_plan* p, const wal_matrix* mats, int n, const int32_t* stage_of,
+bool plan_matches(const wal_body_plan* p, int fmt, const wal_matrix* mats, int n, const int32_t* stage_of,
                   const uint16_t* const* xs, float* const* ys, int M, void* ws, size_t ws_bytes) {
-  if (!p || !p->exec || (int)p->mats.size() != n || p->M != M || p->ws != ws || p->ws_bytes != ws_bytes)
+  if (!p || !p->exec || p->fmt != fmt || (int)p->mats.size() != n || p->M != M || p->ws != ws ||
+      p->ws_bytes != ws_bytes)
     return false;
   for (int i = 0; i < n; ++i)
     if (!same_matrix(p->mats[i], mats[i]) || p->stages[i] != stage_of[i] || p->xs[i] != xs[i] || p->ys[i] != ys[i])
@@ -88,29 +90,17 @@ size_t body_ws_total(int n_mats, int M) {
 
 }  // namespace
 
-extern "C" size_t wal_body_workspace_bytes(const wal_matrix* mats, int n_mats, int M) {
-  if (!mats || n_mats <= 0 || M < 1) return 0;
-  for (int i = 0; i < n_mats; ++i)
-    if (!wal_workspace_bytes(&mats[i], M)) return 0;
-  return body_ws_total(n_mats, M);
-}
+namespace wal {
 
-extern "C" int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n_mats, const int32_t* stage_of,
-                             const uint16_t* const* xs, float* const* ys, int M, void* ws, size_t ws_bytes,
-                             wal_stream_t stream) {
-  if (!plan || !mats || !stage_of || !xs || !ys || n_mats <= 0)
-    return fail(WAL_ERR_ARG, "plan, mats, stage_of, xs and ys are required and n_mats > 0");
-  if (M < 1 || M > WAL_MAX_SMALL_M) return fail(WAL_ERR_SHAPE, "body pass supports 1 <= M <= 16");
-  for (int i = 0; i < n_mats; ++i) {
-    int st = check_product_args(&mats[i], xs[i], M, mats[i].K, ys[i], mats[i].N);
-    if (st) return st;
-    if (i && stage_of[i] < stage_of[i - 1]) return fail(WAL_ERR_ARG, "stage_of must be non-decreasing");
-  }
-  const size_t need = wal_body_workspace_bytes(mats, n_mats, M);
-  if (!ws || ws_bytes < need) return fail(WAL_ERR_WORKSPACE, "body-pass workspace too small");
+size_t body_workspace_total(int n_mats, int M) { return body_ws_total(n_mats, M); }
 
+// A body pass over matrices of one format (kFmtPq2: codes point at PQ2_0
+// block buffers, k = r = 0).  The caller has checked every argument.
+int body_pass_impl(wal_body_plan** plan, int fmt, const wal_matrix* mats, int n_mats, const int32_t* stage_of,
+                   const uint16_t* const* xs, float* const* ys, int M, void* ws, size_t ws_bytes,
+                   cudaStream_t stream) {
   wal_body_plan* p = *plan;
-  if (!plan_matches(p, mats, n_mats, stage_of, xs, ys, M, ws, ws_bytes)) {
+  if (!plan_matches(p, fmt, mats, n_mats, stage_of, xs, ys, M, ws, ws_bytes)) {
     if (!p) {
       p = new wal_body_plan();
       cudaError_t e = cudaStreamCreateWithFlags(&p->capture_stream, cudaStreamNonBlocking);
@@ -125,6 +115,7 @@ extern "C" int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n
     cudaError_t se = cudaStreamSynchronize((cudaStream_t)stream);
     if (se != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("stream synchronize: ") + cudaGetErrorString(se));
     release(p);
+    p->fmt = fmt;
     p->mats.assign(mats, mats + n_mats);
     p->stages.assign(stage_of, stage_of + n_mats);
     p->xs.assign(xs, xs + n_mats);
@@ -151,7 +142,7 @@ extern "C" int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n
       groups[gi].stage = gi == 0 ? 0 : groups[gi - 1].stage + (stage_of[lg.first] != stage_of[lgs[gi - 1].first]);
     }
     StreamLaunch L;
-    int st = plan_launch(groups.data(), (int)groups.size(), true, &L);
+    int st = plan_launch(groups.data(), (int)groups.size(), true, fmt, &L);
     if (st) return st;
     if (L.grid > kMaxCtas) return fail(WAL_ERR_UNSUPPORTED, "more than 1024 SMs");
     const int ng = (int)groups.size();
@@ -170,6 +161,7 @@ extern "C" int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n
     prm.n_groups = ng;
     prm.barrier = reinterpret_cast<unsigned int*>(base + kBarrierOffset);
     prm.status = reinterpret_cast<int32_t*>(base);
+    prm.fmt = fmt;
 
     e = cudaStreamBeginCapture(p->capture_stream, cudaStreamCaptureModeThreadLocal);
     if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("begin capture: ") + cudaGetErrorString(e));
@@ -191,9 +183,34 @@ extern "C" int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n
       return fail(WAL_ERR_CUDA, std::string("graph instantiate: ") + cudaGetErrorString(e));
     }
   }
-  cudaError_t e = cudaGraphLaunch(p->exec, (cudaStream_t)stream);
+  cudaError_t e = cudaGraphLaunch(p->exec, stream);
   if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("graph launch: ") + cudaGetErrorString(e));
   return WAL_OK;
+}
+
+}  // namespace wal
+
+extern "C" size_t wal_body_workspace_bytes(const wal_matrix* mats, int n_mats, int M) {
+  if (!mats || n_mats <= 0 || M < 1) return 0;
+  for (int i = 0; i < n_mats; ++i)
+    if (!wal_workspace_bytes(&mats[i], M)) return 0;
+  return body_ws_total(n_mats, M);
+}
+
+extern "C" int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n_mats, const int32_t* stage_of,
+                             const uint16_t* const* xs, float* const* ys, int M, void* ws, size_t ws_bytes,
+                             wal_stream_t stream) {
+  if (!plan || !mats || !stage_of || !xs || !ys || n_mats <= 0)
+    return fail(WAL_ERR_ARG, "plan, mats, stage_of, xs and ys are required and n_mats > 0");
+  if (M < 1 || M > WAL_MAX_SMALL_M) return fail(WAL_ERR_SHAPE, "body pass supports 1 <= M <= 16");
+  for (int i = 0; i < n_mats; ++i) {
+    int st = check_product_args(&mats[i], xs[i], M, mats[i].K, ys[i], mats[i].N);
+    if (st) return st;
+    if (i && stage_of[i] < stage_of[i - 1]) return fail(WAL_ERR_ARG, "stage_of must be non-decreasing");
+  }
+  const size_t need = wal_body_workspace_bytes(mats, n_mats, M);
+  if (!ws || ws_bytes < need) return fail(WAL_ERR_WORKSPACE, "body-pass workspace too small");
+  return body_pass_impl(plan, kFmtV1, mats, n_mats, stage_of, xs, ys, M, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 extern "C" void wal_body_plan_destroy(wal_body_plan* plan) {

@@ -144,17 +144,19 @@ StreamItem make_item(const wal_matrix* m, const uint16_t* x, float* y) {
 }
 
 // Products of one matrix for activation rows [m0, m0 + count) in one launch
-// (one group: every product shares K).
+// (one group: every product shares K).  fmt kFmtPq2: m->codes is a PQ2_0
+// block buffer and k = r = 0.
 int launch_rows(const wal_matrix* m, const uint16_t* X, int ldx, float* Y, int ldy, int m0, int count,
-                cudaStream_t stream, int32_t* status) {
+                cudaStream_t stream, int32_t* status, int fmt) {
   StreamParams prm = {};
   prm.status = status;
+  prm.fmt = fmt;
   for (int i = 0; i < count; ++i)
     prm.items[i] = make_item(m, X + (size_t)(m0 + i) * ldx, Y + (size_t)(m0 + i) * ldy);
   int st = plan_group(prm.items, count, m->K, &prm.group);
   if (st) return st;
   StreamLaunch L;
-  st = plan_launch(&prm.group, 1, false, &L);
+  st = plan_launch(&prm.group, 1, false, fmt, &L);
   if (st) return st;
   return launch_stream(prm, L, stream);
 }
@@ -196,7 +198,8 @@ extern "C" int wal_gemv(const wal_matrix* m, const uint16_t* x, float* y, void* 
   if (st) return st;
   st = ws_check(ws, ws_bytes, product_ws_bytes(m, 1));
   if (st) return st;
-  return launch_rows(m, x, m->K, y, m->N, 0, 1, (cudaStream_t)stream, reinterpret_cast<int32_t*>(ws_base(ws)));
+  return launch_rows(m, x, m->K, y, m->N, 0, 1, (cudaStream_t)stream, reinterpret_cast<int32_t*>(ws_base(ws)),
+                     kFmtV1);
 }
 
 extern "C" int wal_gemm_small_m(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, int ldy,
@@ -209,7 +212,7 @@ extern "C" int wal_gemm_small_m(const wal_matrix* m, const uint16_t* X, int M, i
   if (M > kMaxItems) return launch_tc(m, X, M, ldx, Y, ldy, ws_base(ws), (cudaStream_t)stream);
   for (int m0 = 0; m0 < M; m0 += kMaxItems) {
     st = launch_rows(m, X, ldx, Y, ldy, m0, std::min(kMaxItems, M - m0), (cudaStream_t)stream,
-                     reinterpret_cast<int32_t*>(ws_base(ws)));
+                     reinterpret_cast<int32_t*>(ws_base(ws)), kFmtV1);
     if (st) return st;
   }
   return WAL_OK;

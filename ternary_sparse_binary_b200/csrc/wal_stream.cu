@@ -73,13 +73,22 @@ constexpr uint32_t kBarrierSpin = 1u << 22;  // polls of the grid-barrier counte
 // per buffer, packed at the buffers' own row pitch; otherwise each row is
 // copied on its own at the fixed pitches below.
 constexpr uint32_t kCodePitch = 1024, kSitePitch = 272, kScalePitch = 144;
+// PQ2_0 rows (34-byte blocks: FP16 scale, then 32 code bytes) arrive as one
+// byte range per chunk (one K-slice) or per row (several K-slices, at this
+// pitch: 32 blocks plus the 16-byte widening at both ends).
+constexpr uint32_t kPq2Block = 34, kPq2Pitch = 1152;
 struct ChunkGeom {
   int rpc;                        // rows per chunk
   uint32_t sites, scales, bytes;  // offsets of the site and scale parts, chunk size
 };
-__host__ __device__ inline ChunkGeom chunk_geom(int rpc) {
+__host__ __device__ inline ChunkGeom chunk_geom(int rpc, int fmt) {
   ChunkGeom c;
   c.rpc = rpc;
+  if (fmt == kFmtPq2) {
+    c.sites = c.scales = 0u;
+    c.bytes = (uint32_t)rpc * kPq2Pitch;
+    return c;
+  }
   c.sites = (uint32_t)rpc * kCodePitch;
   c.scales = c.sites + (uint32_t)rpc * kSitePitch;
   c.bytes = c.scales + (uint32_t)rpc * kScalePitch;
@@ -160,30 +169,32 @@ __device__ __forceinline__ int32_t group_dot(const uint32_t (&wv)[8], const uint
 // that groups land on different banks.
 __host__ __device__ inline uint32_t table_stride(bool signed_table) { return signed_table ? 257u : 129u; }
 
-__host__ __device__ inline uint32_t ring_bytes(int warps, int stages, int rpc) {
-  return (uint32_t)warps * stages * chunk_geom(rpc).bytes;
+__host__ __device__ inline uint32_t ring_bytes(int warps, int stages, int rpc, int fmt) {
+  return (uint32_t)warps * stages * chunk_geom(rpc, fmt).bytes;
 }
 struct ProdState;  // defined below
-__host__ __device__ inline uint32_t area_offset(int warps, int stages, int rpc);
+__host__ __device__ inline uint32_t area_offset(int warps, int stages, int rpc, int fmt);
 
 struct AreaPlan {
   uint32_t table, limbs, part, xgsum, gsc, partz, ubuf, vstage, total;
 };
-// Carve-up of the per-group area (offsets relative to the area base).
-__host__ __device__ inline AreaPlan area_plan(int K, int S, int RB, bool signed_table) {
+// Carve-up of the per-group area (offsets relative to the area base).  A
+// PQ2_0 group has no site table and no WALB2 pair.
+__host__ __device__ inline AreaPlan area_plan(int K, int S, int RB, bool signed_table, int fmt) {
   AreaPlan p;
   uint32_t off = 0;
   auto take = [&](uint32_t bytes) { uint32_t o = off; off = (off + bytes + 15u) & ~15u; return o; };
   const uint32_t G = (uint32_t)K / kGroup;
-  p.table = take(G * table_stride(signed_table) * 4u);
+  const bool v1 = fmt != kFmtPq2;
+  p.table = take(v1 ? G * table_stride(signed_table) * 4u : 0u);
   p.limbs = take(G * kLimbStride * 4u);
   p.part = take((uint32_t)S * RB * 4u);  // one partial per (slice, row)
   p.xgsum = take(G * 4u);
   p.gsc = take(G * 4u);
-  p.partz = take((uint32_t)S * WAL_MAX_RANK * 4u);
-  p.ubuf = take((uint32_t)RB * 4u);
+  p.partz = take(v1 ? (uint32_t)S * WAL_MAX_RANK * 4u : 0u);
+  p.ubuf = take(v1 ? (uint32_t)RB * 4u : 0u);
   // V bit planes of the first P ranks (each of the P phases of a slice takes one): P * K / 8 bytes
-  p.vstage = take((uint32_t)(kMaxWarps / S) * (uint32_t)K / 8u);
+  p.vstage = take(v1 ? (uint32_t)(kMaxWarps / S) * (uint32_t)K / 8u : 0u);
   p.total = off;
   return p;
 }
@@ -239,15 +250,47 @@ __host__ __device__ inline TileRec tile_record(const GroupDesc& g, const StreamI
 __device__ __forceinline__ uint32_t site_bytes(int k) { return (uint32_t)k; }
 __device__ __forceinline__ uint32_t scale_bytes(int k) { return k > 0 ? 4u : 2u; }
 
+// Byte range of PQ2_0 blocks [b0, b0 + nb) widened to 16-byte boundaries
+// (the block buffer is zero-padded to a multiple of 16 bytes, so the widened
+// range stays inside it).
+__device__ __forceinline__ void pq2_range(size_t b0, size_t nb, size_t& a, size_t& e) {
+  a = (b0 * kPq2Block) & ~(size_t)15;
+  e = ((b0 + nb) * kPq2Block + 15) & ~(size_t)15;
+}
+
 // Queue the rows of chunk `chunk` of W into ring slot `sl` with mbarrier
 // `bar`.  Site and scale ranges are widened to 16-byte boundaries (every
 // buffer is zero-padded to a multiple of 16 bytes, so the widened range stays
 // inside).
+template <int FMT>
 __device__ __forceinline__ void issue_chunk(const WarpRing& W, uint32_t sl, uint32_t bar, int chunk,
                                             const ChunkGeom& C) {
   const int i0 = chunk * C.rpc;
   const int un = min(C.rpc, W.nmine - i0);
   if (un <= 0) return;
+  if (FMT == kFmtPq2) {
+    const unsigned char* bbase = reinterpret_cast<const unsigned char*>(W.codes);
+    const size_t G = (size_t)W.G;
+    size_t a, e;
+    if (W.one_slice()) {  // the chunk's rows are one contiguous range
+      pq2_range((size_t)(W.nb + i0) * G, (size_t)un * G, a, e);
+      mbar_arrive_expect_tx(bar, (uint32_t)(e - a));
+      bulk_g2s(sl, bbase + a, (uint32_t)(e - a), bar);
+      return;
+    }
+    const size_t ng = (size_t)W.ngroups();
+    uint32_t bytes = 0;
+    for (int u = 0; u < un; ++u) {
+      pq2_range((size_t)(W.nb + i0 + u) * G + 32 * (size_t)W.s, ng, a, e);
+      bytes += (uint32_t)(e - a);
+    }
+    mbar_arrive_expect_tx(bar, bytes);
+    for (int u = 0; u < un; ++u) {
+      pq2_range((size_t)(W.nb + i0 + u) * G + 32 * (size_t)W.s, ng, a, e);
+      bulk_g2s(sl + (uint32_t)u * kPq2Pitch, bbase + a, (uint32_t)(e - a), bar);
+    }
+    return;
+  }
   const uint32_t kb = site_bytes(W.k), sb = scale_bytes(W.k);
   const unsigned char* cbase = reinterpret_cast<const unsigned char*>(W.codes);
   const unsigned char* abase = reinterpret_cast<const unsigned char*>(W.scales);
@@ -302,8 +345,8 @@ struct ProdState {
   uint32_t slot;      // ring slot of the next chunk to issue (issued mod stages)
   WarpRing W;
 };
-__host__ __device__ inline uint32_t area_offset(int warps, int stages, int rpc) {
-  const uint32_t o = ring_bytes(warps, stages, rpc) + (uint32_t)warps * stages * 8u +
+__host__ __device__ inline uint32_t area_offset(int warps, int stages, int rpc, int fmt) {
+  const uint32_t o = ring_bytes(warps, stages, rpc, fmt) + (uint32_t)warps * stages * 8u +
                      (uint32_t)warps * (uint32_t)((sizeof(ProdState) + 15) & ~(size_t)15);
   return (o + 127u) & ~127u;
 }
@@ -326,11 +369,12 @@ __device__ __forceinline__ void prod_seek(ProdState& ps, const TileRec* sched, i
 // Keep up to `stages` chunks in flight: issue the producer's next chunks (in
 // order, chunk n into slot n mod stages) while fewer are outstanding and, if
 // j_limit >= 0, while they belong to groups up to j_limit.
+template <int FMT>
 __device__ __forceinline__ void prod_topup(ProdState& ps, uint32_t ring, uint32_t mbar, int stages,
                                            const TileRec* sched, int n_groups, const StreamItem* items, int warp,
                                            const ChunkGeom& C, int j_limit) {
   while (ps.j < n_groups && ps.issued - ps.consumed < (uint32_t)stages && (j_limit < 0 || ps.j <= j_limit)) {
-    issue_chunk(ps.W, ring + ps.slot * C.bytes, mbar + ps.slot * 8u, ps.c, C);
+    issue_chunk<FMT>(ps.W, ring + ps.slot * C.bytes, mbar + ps.slot * 8u, ps.c, C);
     ++ps.issued;
     if (++ps.slot == (uint32_t)stages) ps.slot = 0;
     if (++ps.c == ps.nc) {
@@ -386,6 +430,27 @@ __device__ __forceinline__ float row_value(uint32_t crow, uint32_t srow, uint32_
   return fmaf(alpha, (float)tdot, beta * (float)q) * gsc;
 }
 
+// One PQ2_0 row's contribution of this lane's block at shared address A
+// (2-byte aligned): d * T.x over the block's 128 columns.  The block is read
+// as nine aligned words from A rounded down to 4 bytes; each code word is
+// then a byte permute of two neighbours (bytes 2..5 when A is 4-byte
+// aligned, bytes 4..7 when it is not), and d is the block's first two bytes.
+__device__ __forceinline__ float pq2_row_value(uint32_t A, const uint32_t (&lb)[8][kLimbWords], int32_t xs,
+                                               float gsc) {
+  const uint32_t B = A & ~3u;
+  uint32_t w[9];
+#pragma unroll
+  for (int i = 0; i < 9; ++i) w[i] = ptx::lds32(B + 4u * (uint32_t)i);
+  const bool odd = (A & 2u) != 0u;
+  const uint32_t sel = odd ? 0x7654u : 0x5432u;
+  uint32_t wv[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) wv[q] = __byte_perm(w[q], w[q + 1], sel);
+  const uint32_t dbits = __byte_perm(w[0], 0u, odd ? 0x4432u : 0x4410u);
+  const int32_t tdot = group_dot(wv, lb) - xs;
+  return fp16_bits_to_float(dbits) * ((float)tdot * gsc);
+}
+
 // Everything a warp needs to walk its ring.
 struct RingCtx {
   uint32_t ring, mbar;  // this warp's ring slots and mbarriers (shared window)
@@ -436,7 +501,46 @@ __device__ __forceinline__ bool run_rows(const WarpRing& W, const RingCtx& R, ui
     __syncwarp();  // every lane has consumed the slot before it is refilled
     if (lane == 0) {
       ++R.ps->consumed;
-      prod_topup(*R.ps, R.ring, R.mbar, R.stages, R.sched, R.n_groups, R.items, R.warp, C, -1);
+      prod_topup<kFmtV1>(*R.ps, R.ring, R.mbar, R.stages, R.sched, R.n_groups, R.items, R.warp, C, -1);
+    }
+    if (++st == (uint32_t)R.stages) {
+      st = 0;
+      parity ^= 1u;
+    }
+  }
+  return true;
+}
+
+// run_rows for PQ2_0 rows: lane l takes block l of the warp's K-slice.
+__device__ __forceinline__ bool run_rows_pq2(const WarpRing& W, const RingCtx& R, uint32_t& st, uint32_t& parity,
+                                             int RB, int lane, bool active, const uint32_t (&lb)[8][kLimbWords],
+                                             int32_t xs, float gsc, float* part) {
+  const ChunkGeom& C = R.C;
+  const int nc = (W.nmine + C.rpc - 1) / C.rpc;
+  float* mine = part + W.s * RB + W.r0;
+  const bool one = W.one_slice();
+  const uint32_t G = (uint32_t)W.G, rowb = G * kPq2Block;
+#pragma unroll 1
+  for (int j = 0; j < nc; ++j) {
+    const uint32_t sl = R.ring + st * C.bytes;
+    if (!mbar_wait(R.mbar + st * 8u, parity, R.status)) return false;
+#pragma unroll
+    for (int u = 0; u < kMaxRowsPerChunk; ++u) {
+      const int i = j * C.rpc + u;
+      if (u < C.rpc && i < W.nmine) {  // uniform across the warp
+        // where the widened copy put the row (only the low 4 bits of the byte offset matter)
+        const uint32_t row = one ? sl + (((uint32_t)(W.nb + j * C.rpc) * rowb) & 15u) + (uint32_t)u * rowb
+                                 : sl + (uint32_t)u * kPq2Pitch +
+                                       ((((uint32_t)(W.nb + i) * G + 32u * (uint32_t)W.s) * kPq2Block) & 15u);
+        const float v = pq2_row_value(row + kPq2Block * (uint32_t)lane, lb, xs, gsc);
+        const float tot = warp_sum(active ? v : 0.f);
+        if (lane == 0) mine[i] = tot;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      ++R.ps->consumed;
+      prod_topup<kFmtPq2>(*R.ps, R.ring, R.mbar, R.stages, R.sched, R.n_groups, R.items, R.warp, C, -1);
     }
     if (++st == (uint32_t)R.stages) {
       st = 0;
@@ -456,7 +560,9 @@ __device__ __forceinline__ void load_x(const uint16_t* x, int K, uint4 (&xr)[kMa
   }
 }
 
-template <bool SIGNED_TABLE>
+// PQ2 = true: no site table, and the limb image keeps every group in natural
+// word order (PQ2_0 code words are read one by one, not as 16-byte halves).
+template <bool SIGNED_TABLE, bool PQ2>
 __device__ __forceinline__ void build_image(const uint4 (&xr)[kMaxXChunks], int K, unsigned char* area,
                                             const AreaPlan& ap) {
   const int threads = blockDim.x, tid = threadIdx.x, lane = tid & 31;
@@ -504,7 +610,7 @@ __device__ __forceinline__ void build_image(const uint4 (&xr)[kMaxXChunks], int 
     // A group read by a lane with bit 2 set is stored with its halves swapped
     // (words 0-3 <-> 4-7), the order in which that lane holds its limbs, so
     // that every lane reads its image front to back without bank conflicts.
-    const int wl = ((c >> 4) & 7) ^ ((gg & 4) ? 4 : 0);
+    const int wl = ((c >> 4) & 7) ^ ((!PQ2 && (gg & 4)) ? 4 : 0);
     uint16_t* img16 = reinterpret_cast<uint16_t*>(limbs + (size_t)gg * kLimbStride);
 #pragma unroll
     for (int L2 = 0; L2 < 3; ++L2)
@@ -517,11 +623,13 @@ __device__ __forceinline__ void build_image(const uint4 (&xr)[kMaxXChunks], int 
       gsc_s[gg] = emax >= 22u ? __uint_as_float((emax - 21u) << 23) : __uint_as_float(1u << (emax + 1u));
     }
     // site table: entry e of group gg (e = site byte) at gg * stride + e
-    int32_t* trow = table + (size_t)gg * tstride + pos;
+    if (!PQ2) {
+      int32_t* trow = table + (size_t)gg * tstride + pos;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      trow[q] = X[q];
-      if (SIGNED_TABLE) trow[128 + q] = -X[q];
+      for (int q = 0; q < 8; ++q) {
+        trow[q] = X[q];
+        if (SIGNED_TABLE) trow[128 + q] = -X[q];
+      }
     }
   }
   __syncthreads();
@@ -533,7 +641,7 @@ __device__ __forceinline__ void prefetch_l1(const void* p) {
 
 // One group on this CTA (which owns the tile t of it).  Returns false (on
 // every thread) when some wait of the CTA gave up.
-template <bool SIGNED_TABLE>
+template <int FMT, bool SIGNED_TABLE>
 __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int j, uint32_t& st, uint32_t& parity,
                                          unsigned char* area, float* s_z) {
   const int threads = blockDim.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -541,9 +649,10 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
   const StreamItem& it = R.items[t.item];
   WarpRing W;
   warp_work(t, &it, warp, W);
-  const int r = it.r, ks = it.k;
+  constexpr bool PQ2 = FMT == kFmtPq2;
+  const int r = PQ2 ? 0 : it.r, ks = PQ2 ? 0 : it.k;
   const bool worker = warp < S * P;
-  const AreaPlan ap = area_plan(K, S, RB, SIGNED_TABLE);
+  const AreaPlan ap = area_plan(K, S, RB, SIGNED_TABLE, FMT);
   float* partz = reinterpret_cast<float*>(area + ap.partz);
   float* part = reinterpret_cast<float*>(area + ap.part);
   uint32_t* ubuf = reinterpret_cast<uint32_t*>(area + ap.ubuf);
@@ -566,7 +675,7 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
     const TileRec tn = R.sched[j + 1 + tid];
     if (tn.rows) prefetch_l1(R.items + tn.item);
   }
-  build_image<SIGNED_TABLE>(xr, K, area, ap);
+  build_image<SIGNED_TABLE, PQ2>(xr, K, area, ap);
 
   // the 96 limb words of this lane's group into registers; on lanes with bit
   // 2 set register word w holds group word w ^ 4 (stored so in the image), as
@@ -620,7 +729,9 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
     }
   const uint32_t tab = ptx::smem_u32(area + ap.table) + (uint32_t)g * table_stride(SIGNED_TABLE) * 4u;
   bool ok = true;
-  if (worker) {
+  if (PQ2) {
+    if (worker) ok = run_rows_pq2(W, R, st, parity, RB, lane, active, lb, xs, gsc, part);
+  } else if (worker) {
     switch (ks) {
       case 8: ok = run_rows<8, SIGNED_TABLE>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
       case 4: ok = run_rows<4, SIGNED_TABLE>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
@@ -630,7 +741,7 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
   }
 
   // keep this warp's ring full (a warp with no rows here has issued nothing since the first fill)
-  if (lane == 0) prod_topup(*R.ps, R.ring, R.mbar, R.stages, R.sched, R.n_groups, R.items, R.warp, R.C, -1);
+  if (lane == 0) prod_topup<FMT>(*R.ps, R.ring, R.mbar, R.stages, R.sched, R.n_groups, R.items, R.warp, R.C, -1);
   // the last warp (fewest rows) warms L2 with the x of the CTA's next tile
   if (warp == (int)(blockDim.x / 32) - 1 && lane == 0)
     for (int jn = j + 1; jn < R.n_groups; ++jn) {
@@ -681,6 +792,7 @@ __device__ __forceinline__ void grid_barrier(unsigned int* ctr, unsigned int tar
   __syncthreads();
 }
 
+template <int FMT>
 __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_constant__ StreamParams prm) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ float s_z[WAL_MAX_RANK];
@@ -703,10 +815,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
 
   RingCtx R;
   const uint32_t base = ptx::smem_u32(smem);
-  R.C = chunk_geom(prm.rpc);
+  R.C = chunk_geom(prm.rpc, FMT);
   R.ring = base + (uint32_t)warp * stages * R.C.bytes;
-  R.mbar = base + ring_bytes(warps, stages, prm.rpc) + (uint32_t)warp * stages * 8u;
-  R.ps = reinterpret_cast<ProdState*>(smem + ring_bytes(warps, stages, prm.rpc) + (uint32_t)warps * stages * 8u +
+  R.mbar = base + ring_bytes(warps, stages, prm.rpc, FMT) + (uint32_t)warp * stages * 8u;
+  R.ps = reinterpret_cast<ProdState*>(smem + ring_bytes(warps, stages, prm.rpc, FMT) + (uint32_t)warps * stages * 8u +
                                       (uint32_t)warp * (uint32_t)((sizeof(ProdState) + 15) & ~(size_t)15));
   R.stages = stages;
   R.sched = sched;
@@ -727,7 +839,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
     // run-ahead into later groups starts once that group is under way
     int j0 = 0;
     while (j0 + 1 < n_groups && sched[j0].rows == 0) ++j0;
-    prod_topup(*R.ps, R.ring, R.mbar, stages, sched, n_groups, items, warp, R.C, j0);
+    prod_topup<FMT>(*R.ps, R.ring, R.mbar, stages, sched, n_groups, items, warp, R.C, j0);
   }
   __syncwarp();
 
@@ -742,8 +854,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
       grid_barrier(prm.barrier, nbar * gridDim.x, prm.status);
     }
     if (t.rows == 0 || dead) continue;  // uniform across the CTA
-    const bool ok = t.signed_table ? do_group<true>(t, R, j, st, parity, area, s_z)
-                                   : do_group<false>(t, R, j, st, parity, area, s_z);
+    bool ok;
+    if (FMT == kFmtPq2) ok = do_group<kFmtPq2, false>(t, R, j, st, parity, area, s_z);
+    else ok = t.signed_table ? do_group<kFmtV1, true>(t, R, j, st, parity, area, s_z)
+                             : do_group<kFmtV1, false>(t, R, j, st, parity, area, s_z);
     dead = !ok;
   }
   // never leave with bulk copies in flight: after a wait gave up, wait
@@ -776,7 +890,9 @@ int stream_init() {
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&g_max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, g_max_smem - 1024);
+      e = cudaFuncSetAttribute(stream_kernel<kFmtV1>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_max_smem - 1024);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(stream_kernel<kFmtPq2>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_max_smem - 1024);
     g_err = e;
   });
   if (g_err != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("device initialisation: ") + cudaGetErrorString(g_err));
@@ -821,7 +937,7 @@ int plan_group(StreamItem* items, int n, int K, GroupDesc* out) {
   return WAL_OK;
 }
 
-int plan_launch(GroupDesc* groups, int n_groups, bool persistent, StreamLaunch* out) {
+int plan_launch(GroupDesc* groups, int n_groups, bool persistent, int fmt, StreamLaunch* out) {
   StreamLaunch L = {};
   int warps = 0;
   for (int j = 0; j < n_groups; ++j) warps = std::max(warps, groups[j].S * groups[j].P);
@@ -833,13 +949,13 @@ int plan_launch(GroupDesc* groups, int n_groups, bool persistent, StreamLaunch* 
   static const int kRing[6][2] = {{3, 4}, {3, 3}, {2, 4}, {3, 2}, {2, 3}, {2, 2}};
   for (const auto& rs : kRing) {
     const int rpc = rs[0], stages = rs[1];
-    const uint32_t soff = area_offset(warps, stages, rpc);
+    const uint32_t soff = area_offset(warps, stages, rpc, fmt);
     const uint32_t off = soff + sched_bytes;
     uint32_t need = off;
     bool fits = true;
     for (int j = 0; j < n_groups && fits; ++j) {
       const GroupDesc& g = groups[j];
-      const uint32_t as = area_plan(g.K, g.S, g.RB, true).total, au = area_plan(g.K, g.S, g.RB, false).total;
+      const uint32_t as = area_plan(g.K, g.S, g.RB, true, fmt).total, au = area_plan(g.K, g.S, g.RB, false, fmt).total;
       if (off + as <= limit) need = std::max(need, off + as);
       else if (off + au <= limit) need = std::max(need, off + au);
       else fits = false;
@@ -847,7 +963,7 @@ int plan_launch(GroupDesc* groups, int n_groups, bool persistent, StreamLaunch* 
     if (!fits) continue;
     for (int j = 0; j < n_groups; ++j) {
       const GroupDesc& g = groups[j];
-      groups[j].signed_table = off + area_plan(g.K, g.S, g.RB, true).total <= limit ? 1 : 0;
+      groups[j].signed_table = fmt == kFmtV1 && off + area_plan(g.K, g.S, g.RB, true, fmt).total <= limit ? 1 : 0;
     }
     L.stages = stages;
     L.rpc = rpc;
@@ -882,7 +998,8 @@ static int launch(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream,
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = cooperative ? 1 : 0;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, stream_kernel, prm);
+  const cudaError_t e = prm.fmt == kFmtPq2 ? cudaLaunchKernelEx(&cfg, stream_kernel<kFmtPq2>, prm)
+                                            : cudaLaunchKernelEx(&cfg, stream_kernel<kFmtV1>, prm);
   if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("stream_kernel launch: ") + cudaGetErrorString(e));
   return WAL_OK;
 }
@@ -898,7 +1015,9 @@ int launch_stream(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream)
 int launch_body(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream) {
   if (!prm.t_sched || !prm.t_items || !prm.barrier) return fail(WAL_ERR_ARG, "body launch without tables");
   int per_sm = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, stream_kernel, L.threads, L.smem);
+  cudaError_t e = prm.fmt == kFmtPq2
+                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, stream_kernel<kFmtPq2>, L.threads, L.smem)
+                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, stream_kernel<kFmtV1>, L.threads, L.smem);
   if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("occupancy query: ") + cudaGetErrorString(e));
   if (per_sm < 1 || L.grid > per_sm * num_sms())
     return fail(WAL_ERR_UNSUPPORTED, "the persistent launch does not fit on the device at once");

@@ -9,6 +9,12 @@ namespace wal {
 
 constexpr int kMaxItems = 16;
 
+// Weight formats a launch can stream (one per launch):
+//  kFmtV1  layout v1 of the direct-packed product (codes, sites, scales, WALB2);
+//  kFmtPq2 PQ2_0 plain-ternary blocks (FP16 scale + 32 code bytes per 128
+//          weights); `codes` then points at the block buffer, k = r = 0.
+enum : int { kFmtV1 = 0, kFmtPq2 = 1 };
+
 // One product y = W x.
 struct StreamItem {
   const uint32_t* codes;
@@ -58,6 +64,7 @@ struct StreamParams {
   uint32_t area_off;          // shared-memory offset of the per-group area
   unsigned int* barrier;      // grid-barrier counter (zeroed before the launch), body pass only
   int32_t* status;            // workspace status word (may be NULL)
+  int fmt;                    // kFmtV1 or kFmtPq2
 };
 
 struct StreamLaunch {
@@ -73,8 +80,8 @@ int stream_init();
 int num_sms();
 // Fill the geometry of group `g` (K, items) and return WAL_OK or an error.
 int plan_group(StreamItem* items, int n, int K, GroupDesc* g);
-// Shared memory and ring depth for a list of groups.
-int plan_launch(GroupDesc* groups, int n_groups, bool persistent, StreamLaunch* out);
+// Shared memory and ring depth for a list of groups of format `fmt`.
+int plan_launch(GroupDesc* groups, int n_groups, bool persistent, int fmt, StreamLaunch* out);
 // Single group, items inline.
 int launch_stream(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream);
 // Body pass: group and item tables already in device memory; cooperative launch.

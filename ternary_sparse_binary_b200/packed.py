@@ -5,7 +5,7 @@ import numpy as np
 import torch
 
 from . import _abi
-from ._abi import wal_matrix
+from ._abi import wal_matrix, wal_pq2_matrix
 
 
 def _ptr(a):
@@ -52,6 +52,32 @@ class PackedMatrix:
         return _abi.wal_workspace_bytes(self.desc, M)
 
 
+def pack_pq2_host(T, d, N, K):
+    """Pack T (int8 [N, K]) and d (fp16 bits [N, K/128]) into a PQ2_0 buffer
+    with the library's host packer; returns a numpy uint8 array."""
+    out = np.empty(_abi.wal_pq2_bytes(N, K), dtype=np.uint8)
+    T = np.ascontiguousarray(T, np.int8)
+    d = np.ascontiguousarray(d, np.uint16)
+    _abi.wal_pq2_pack(_ptr(T), _ptr(d), N, K, _ptr(out))
+    return out
+
+
+class Pq2Matrix:
+    """A PQ2_0 block buffer on a CUDA device plus its wal_pq2_matrix descriptor."""
+
+    def __init__(self, buf, N, K, device="cuda"):
+        self.N, self.K = N, K
+        self.buf = torch.from_numpy(np.ascontiguousarray(buf).view(np.uint8).reshape(-1)).to(device)
+        self.desc = wal_pq2_matrix(N, K, self.buf.data_ptr())
+
+    @property
+    def nbytes(self):
+        return self.buf.numel()
+
+    def workspace_bytes(self, M=1):
+        return _abi.wal_pq2_workspace_bytes(self.desc, M)
+
+
 def to_device(bufs, N, K, k, r, device="cuda"):
     return PackedMatrix(bufs, N, K, k, r, device)
 
@@ -62,21 +88,25 @@ def _stream_handle(stream=None):
 
 
 class BodyPass:
-    """Owns a wal_body_plan handle and its workspace; run() replays the graph."""
+    """Owns a wal_body_plan handle and its workspace; run() replays the graph.
+    The matrices are all PackedMatrix (layout v1) or all Pq2Matrix (PQ2_0)."""
 
     def __init__(self, mats, stage_of, xs, ys, M=1, device="cuda"):
         self.mats = list(mats)
         self.descs = [m.desc for m in self.mats]
+        self.pq2 = isinstance(self.mats[0], Pq2Matrix)
+        if any(isinstance(m, Pq2Matrix) != self.pq2 for m in self.mats):
+            raise ValueError("a body pass takes matrices of one format")
         self.stage_of = [int(s) for s in stage_of]
         self.xs, self.ys, self.M = list(xs), list(ys), M
-        nb = _abi.wal_body_workspace_bytes(self.descs, M)
+        nb = (_abi.wal_pq2_body_workspace_bytes if self.pq2 else _abi.wal_body_workspace_bytes)(self.descs, M)
         if nb == 0:
             raise _abi.WalError(_abi.WAL_ERR_ARG, "wal_body_workspace_bytes")
         self.ws = torch.empty(nb, dtype=torch.uint8, device=device)
         self.plan = ctypes.c_void_p(None)
 
     def run(self, stream=None):
-        _abi.wal_body_pass(self.plan, self.descs, self.stage_of, [x.data_ptr() for x in self.xs],
+        (_abi.wal_pq2_body_pass if self.pq2 else _abi.wal_body_pass)(self.plan, self.descs, self.stage_of, [x.data_ptr() for x in self.xs],
                            [y.data_ptr() for y in self.ys], self.M, self.ws.data_ptr(), self.ws.numel(),
                            _stream_handle(stream))
 

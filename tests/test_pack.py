@@ -88,3 +88,31 @@ def test_pack_rejects_null_buffers():
         wal.wal_pack_matrix(c.T.ctypes.data, None, None, c.alpha.ctypes.data, None, None, None, None,
                             4, 256, 4, 2, [None] * 6)
     assert e.value.status == wal.WAL_ERR_ARG
+
+
+# ---------------------------------------------------------------------------
+# PQ2_0 block format
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K", [(1, 128), (3, 256), (64, 4096), (5, 12288), (7, 1152), (33, 5120)])
+def test_pq2_pack_matches_oracle_bytes(N, K):
+    from oracle import pq2_oracle as pq
+    from wal_synth import gen_pq2
+    T, d = gen_pq2(N, K, 83, N + K)
+    mine = wal.pack_pq2_host(T, d, N, K)
+    assert mine.size == pq.packed_bytes(N, K) == wal.wal_pq2_bytes(N, K)
+    assert np.array_equal(mine, pq.pack(pq.Pq2(N, K, T, d)))
+
+
+def test_pq2_pack_rejects_bad_trit():
+    T = np.zeros((1, 128), np.int8)
+    T[0, 7] = 2
+    with pytest.raises(wal.WalError) as e:
+        wal.pack_pq2_host(T, np.zeros((1, 1), np.uint16), 1, 128)
+    assert e.value.status == wal.WAL_ERR_FORMAT
+
+
+def test_pq2_sizes_reject_bad_shape():
+    assert wal.wal_pq2_bytes(4, 100) == 0
+    assert wal.wal_pq2_bytes(0, 128) == 0
+    assert wal.wal_pq2_bytes(2, 128) == 80
