@@ -22,6 +22,7 @@ from .gen import (  # noqa: F401
     config_plan,
     gen_matrix,
     gen_pq2,
+    gen_base3,
     workload_id,
     WORKLOAD_IDS,
     CONFIG_SEED,

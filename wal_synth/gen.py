@@ -240,3 +240,13 @@ def gen_pq2(N: int, K: int, config_id: int = 0, matrix_index: int = 0):
     Returns (T int8 [N, K], d uint16 fp16 bits [N, K/128])."""
     c = gen_components(N, K, 0, 0, config_id, matrix_index)
     return c.T, c.alpha
+
+
+def gen_base3(N: int, K: int, config_id: int = 0, matrix_index: int = 0):
+    """One plain-ternary matrix for the base-3 container: T iid as in
+    gen_components and one BF16 scale per (row, 128-group), bf16(|N(0, 0.02)|).
+    Returns (T int8 [N, K], s uint16 bf16 bits [N, K/128])."""
+    c = gen_components(N, K, 0, 0, config_id, matrix_index)
+    rs = rng_for(config_id, matrix_index, S_SCALES)
+    s = bf16_bits_from_f32(np.abs(rs.normal(0.0, 0.02, size=(N, K // GROUP))).astype(np.float32))
+    return c.T, s
