@@ -220,6 +220,36 @@ int wal_pq2_body_pass(wal_body_plan** plan, const wal_pq2_matrix* mats, int n_ma
                       const uint16_t* const* xs, float* const* ys, int M, void* ws, size_t ws_bytes,
                       wal_stream_t stream);
 
+/* ---- the base-3 container and its conversion (the prepare step) -----------
+ * The WAL2-Ternary-27B card (section on bit widths) keeps its canonical
+ * ternary base five trits to a byte (8 / 5 = 1.6 bits per symbol) with a
+ * BF16 scale per 128 weights.  This library's reading of the bytes: byte m
+ * of a row holds trits 5m .. 5m + 4 as sum_i (t_i + 1) * 3^i (trit 5m + i is
+ * digit i, least significant first); values 243..255 are invalid; each row
+ * starts on a byte (ceil(K / 5) bytes per row, rows back to back); digits
+ * past a row's last trit are 0; the buffer is zero-padded to 16 bytes.
+ * Scales: bf16 bits [N][K/128]. */
+
+/* Bytes of the base-3 buffer of an N x K matrix; 0 on a bad shape. */
+size_t wal_base3_bytes(int N, int K);
+
+/* Pack T [N][K] int8 in {-1,0,1} into the base-3 buffer `out` (host memory,
+ * wal_base3_bytes(N, K) bytes, padding zeroed).  Host only, multi-threaded.
+ * WAL_ERR_FORMAT when T leaves {-1,0,1}. */
+int wal_base3_pack(const int8_t* T, int N, int K, void* out);
+
+/* The prepare step on the GPU: base-3 bytes b3 and BF16 scales [N][K/128]
+ * become the layout-v1 code plane `codes` (uint32 [N][K/16], code c = t + 1)
+ * and the k = 0 scale plane `alpha` (fp16 bits [N][K/128], BF16 rounded to
+ * nearest even; its 16-byte padding is zeroed).  All device pointers,
+ * 16-byte aligned; output sizes as wal_packed_sizes(N, K, 0, r) gives for
+ * buffers 0 and 2.  ws: at least 512 bytes.  Synchronises `stream` and
+ * returns WAL_ERR_FORMAT when a byte is above 242, a digit past a row's end
+ * is nonzero, or a scale is not finite or overflows FP16 (the outputs are
+ * then incomplete). */
+int wal_base3_convert(const uint8_t* b3, const uint16_t* scales_bf16, int N, int K, uint32_t* codes,
+                      uint16_t* alpha, void* ws, size_t ws_bytes, wal_stream_t stream);
+
 const char* wal_status_string(int status);
 const char* wal_last_error(void);
 

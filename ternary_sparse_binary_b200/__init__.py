@@ -14,5 +14,6 @@ from ._abi import (  # noqa: F401
     wal_body_plan_destroy, wal_status_string, wal_last_error,
     wal_pq2_matrix, wal_pq2_bytes, wal_pq2_pack, wal_pq2_workspace_bytes, wal_pq2_gemm,
     wal_pq2_body_workspace_bytes, wal_pq2_body_pass,
+    wal_base3_bytes, wal_base3_pack, wal_base3_convert,
 )
 from .packed import PackedMatrix, Pq2Matrix, pack_host, pack_pq2_host, to_device, BodyPass  # noqa: F401

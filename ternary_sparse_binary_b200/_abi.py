@@ -27,6 +27,7 @@ EXPORTED_SYMBOLS = [
     "wal_body_workspace_bytes", "wal_body_pass", "wal_body_plan_destroy",
     "wal_pq2_bytes", "wal_pq2_pack", "wal_pq2_workspace_bytes", "wal_pq2_gemm",
     "wal_pq2_body_workspace_bytes", "wal_pq2_body_pass",
+    "wal_base3_bytes", "wal_base3_pack", "wal_base3_convert",
     "wal_status_string", "wal_last_error",
 ]
 
@@ -87,6 +88,10 @@ lib.wal_pq2_body_workspace_bytes.argtypes = [_PP, _i, _i]
 lib.wal_pq2_body_workspace_bytes.restype = _sz
 lib.wal_pq2_body_pass.argtypes = [ctypes.POINTER(_vp), _PP, _i, ctypes.POINTER(ctypes.c_int32),
                                   ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp, _sz, _vp]
+lib.wal_base3_bytes.argtypes = [_i, _i]
+lib.wal_base3_bytes.restype = _sz
+lib.wal_base3_pack.argtypes = [_vp, _i, _i, _vp]
+lib.wal_base3_convert.argtypes = [_vp, _vp, _i, _i, _vp, _vp, _vp, _sz, _vp]
 lib.wal_status_string.argtypes = [_i]
 lib.wal_status_string.restype = ctypes.c_char_p
 lib.wal_last_error.argtypes = []
@@ -199,3 +204,16 @@ def wal_pq2_body_pass(plan, mats, stage_of, xs, ys, M, ws, ws_bytes, stream):
     yarr = (_vp * n)(*ys)
     return _check(lib.wal_pq2_body_pass(ctypes.byref(plan), marr, n, sarr, xarr, yarr, M, ws, ws_bytes,
                                         stream), "wal_pq2_body_pass")
+
+
+def wal_base3_bytes(N, K):
+    return int(lib.wal_base3_bytes(N, K))
+
+
+def wal_base3_pack(T, N, K, out):
+    return _check(lib.wal_base3_pack(T, N, K, out), "wal_base3_pack")
+
+
+def wal_base3_convert(b3, scales_bf16, N, K, codes, alpha, ws, ws_bytes, stream):
+    return _check(lib.wal_base3_convert(b3, scales_bf16, N, K, codes, alpha, ws, ws_bytes, stream),
+                  "wal_base3_convert")

@@ -116,3 +116,24 @@ def test_pq2_sizes_reject_bad_shape():
     assert wal.wal_pq2_bytes(4, 100) == 0
     assert wal.wal_pq2_bytes(0, 128) == 0
     assert wal.wal_pq2_bytes(2, 128) == 80
+
+
+# ---------------------------------------------------------------------------
+# base-3 container
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K", [(1, 128), (2, 256), (3, 384), (4, 512), (5, 640), (2, 4096), (1, 17408)])
+def test_base3_pack_matches_oracle_bytes(N, K):
+    from oracle import base3_oracle as b3
+    from wal_synth import gen_base3
+    T, _ = gen_base3(N, K, 84, N + K)
+    out = np.empty(wal.wal_base3_bytes(N, K), np.uint8)
+    wal.wal_base3_pack(T.ctypes.data, N, K, out.ctypes.data)
+    assert out.size == b3.packed_bytes(N, K)
+    assert np.array_equal(out, b3.pack(T))
+
+
+def test_base3_sizes():
+    assert wal.wal_base3_bytes(1, 128) == 32  # 26 bytes, padded
+    assert wal.wal_base3_bytes(2, 5120) == 2048
+    assert wal.wal_base3_bytes(1, 100) == 0
