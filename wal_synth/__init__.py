@@ -23,6 +23,8 @@ from .gen import (  # noqa: F401
     gen_matrix,
     gen_pq2,
     gen_base3,
+    gen_rc1,
+    f24_bytes_from_f32,
     workload_id,
     WORKLOAD_IDS,
     CONFIG_SEED,

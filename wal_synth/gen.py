@@ -250,3 +250,36 @@ def gen_base3(N: int, K: int, config_id: int = 0, matrix_index: int = 0):
     rs = rng_for(config_id, matrix_index, S_SCALES)
     s = bf16_bits_from_f32(np.abs(rs.normal(0.0, 0.02, size=(N, K // GROUP))).astype(np.float32))
     return c.T, s
+
+
+S_LOWRANK2 = 6  # stream of the second WALB2 path of an RC1 matrix
+
+
+def f24_bytes_from_f32(a) -> np.ndarray:
+    """Round float32 values to the 24-bit float storage type (the upper three
+    bytes of an FP32, round to nearest, ties to even); uint8 [..., 3] little endian."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7F + ((u >> 8) & 1)) >> 8).astype(np.uint32)
+    return np.stack([(r >> (8 * i)) & 0xFF for i in range(3)], axis=-1).astype(np.uint8)
+
+
+def gen_rc1(N: int, K: int, k: int, r1: int, r2: int, config_id: int = 0, matrix_index: int = 0):
+    """One RC1-format matrix: T and sites as in gen_components; alpha, beta
+    (|N(0, 0.02)|, |N(0, 0.005)|) and the per-rank scales (|N(0, 0.01)|) rounded
+    to 24-bit floats; two WALB2 paths of ranks r1 and r2 with iid +-1 U, V.
+    Returns a dict of arrays (T, site_pos, site_sign, alpha24, beta24, U1, V1,
+    s1, U2, V2, s2) plus N, K, k."""
+    G = K // GROUP
+    c = gen_components(N, K, k, 0, config_id, matrix_index)
+    rs = rng_for(config_id, matrix_index, S_SCALES)
+    alpha = f24_bytes_from_f32(np.abs(rs.normal(0.0, 0.02, size=(N, G))).astype(np.float32))
+    beta = f24_bytes_from_f32(np.abs(rs.normal(0.0, 0.005, size=(N, G))).astype(np.float32))
+    paths = []
+    for stream, r in ((S_LOWRANK, r1), (S_LOWRANK2, r2)):
+        rl = rng_for(config_id, matrix_index, stream)
+        U = (rl.integers(0, 2, size=(N, r), dtype=np.int8) * 2 - 1).astype(np.int8)
+        V = (rl.integers(0, 2, size=(K, r), dtype=np.int8) * 2 - 1).astype(np.int8)
+        s = f24_bytes_from_f32(np.abs(rl.normal(0.0, 0.01, size=r)).astype(np.float32)).reshape(r, 3)
+        paths += [U, V, s]
+    return dict(N=N, K=K, k=k, T=c.T, site_pos=c.site_pos, site_sign=c.site_sign, alpha24=alpha, beta24=beta,
+                U1=paths[0], V1=paths[1], s1=paths[2], U2=paths[3], V2=paths[4], s2=paths[5])
