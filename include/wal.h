@@ -250,6 +250,58 @@ int wal_base3_pack(const int8_t* T, int N, int K, void* out);
 int wal_base3_convert(const uint8_t* b3, const uint16_t* scales_bf16, int N, int K, uint32_t* codes,
                       uint16_t* alpha, void* ws, size_t ws_bytes, wal_stream_t stream);
 
+/* ---- RC1 storage: 24-bit float scales and two WALB2 paths ------------------
+ * The WAL-Ternary-27B-RC1 card ("Representation") keeps the body scales in a
+ * 24-bit float format that its prepared compute cache expands to FP32, and
+ * WALB2 as two packed binary low-rank paths:
+ *   W = alpha (x) T + beta (x) R + U1 diag(s1) V1^T + U2 diag(s2) V2^T.
+ * This library's reading (the card's storage ABI is not among its pages):
+ * a 24-bit float is the upper three bytes of an IEEE FP32, little endian;
+ * alpha, beta, s1 and s2 use it; the canonical planes are
+ *   scales24 uint8 [N][G][2][3] ({alpha, beta}) when k > 0, [N][G][3] when k = 0;
+ *   u_p uint32 [N][ceil(r_p/32)], v_p uint32 [r_p][K/32] (set bit = -1),
+ *   s_p uint8 [r_p][3];  r1 + r2 <= 32;
+ * each zero-padded to 16 bytes (wal_rc1_sizes).  The prepared matrix is
+ * layout v1 with FP32 in place of FP16: scales float {alpha, beta} [N][G]
+ * (alpha [N][G] when k = 0), one rank block r = r1 + r2 with path 1's ranks
+ * first, lr_scale float [r]. */
+typedef struct wal_rc1_matrix {  /* a prepared RC1 matrix; device pointers, 16-byte aligned */
+  int32_t N, K, k, r;
+  const uint32_t* codes;         /* layout v1 code plane */
+  const uint8_t* sites;          /* layout v1 site bytes (NULL when k == 0) */
+  const float* scales;           /* FP32 {alpha, beta} [N][G], or alpha [N][G] when k == 0 */
+  const uint32_t* u_bits;        /* [N][ceil(r/32)] */
+  const uint32_t* v_bits;        /* [r][K/32] */
+  const float* lr_scale;         /* FP32 [r] */
+} wal_rc1_matrix;
+
+/* Byte sizes of the canonical RC1 planes (scales24, u1, v1, s1, u2, v2, s2)
+ * and of the prepared planes (scales32, u_bits, v_bits, lr32).  Host only.
+ * WAL_ERR_SHAPE on a bad shape or r1 + r2 > 32. */
+int wal_rc1_sizes(int N, int K, int k, int r1, int r2, size_t canonical[7], size_t prepared[4]);
+
+/* The prepare step on the GPU: decode every 24-bit scale to FP32 and merge
+ * the two paths into one rank block (U words: path 2's bits shifted up by
+ * r1; V bit rows and per-rank scales concatenated, path 1 first).  Device
+ * pointers, 16-byte aligned; a path with r_p = 0 may pass NULL buffers.  The
+ * code plane and the site bytes are layout v1 already and are used as they
+ * are.  Asynchronous. */
+int wal_rc1_prepare(int N, int K, int k, const uint8_t* scales24, int r1, const uint32_t* u1, const uint32_t* v1,
+                    const uint8_t* s1_24, int r2, const uint32_t* u2, const uint32_t* v2, const uint8_t* s2_24,
+                    float* scales32, uint32_t* u_bits, uint32_t* v_bits, float* lr32, wal_stream_t stream);
+
+/* Products of a prepared RC1 matrix, 1 <= M <= 16, with the same contract as
+ * wal_gemm_small_m (the FP32-scale specialisation of the decode-GEMV), and
+ * the body pass over prepared RC1 matrices with the contract of
+ * wal_body_pass. */
+size_t wal_rc1_workspace_bytes(const wal_rc1_matrix* m, int M);
+int wal_rc1_gemm(const wal_rc1_matrix* m, const uint16_t* X, int M, int ldx, float* Y, int ldy, void* ws,
+                 size_t ws_bytes, wal_stream_t stream);
+size_t wal_rc1_body_workspace_bytes(const wal_rc1_matrix* mats, int n_mats, int M);
+int wal_rc1_body_pass(wal_body_plan** plan, const wal_rc1_matrix* mats, int n_mats, const int32_t* stage_of,
+                      const uint16_t* const* xs, float* const* ys, int M, void* ws, size_t ws_bytes,
+                      wal_stream_t stream);
+
 const char* wal_status_string(int status);
 const char* wal_last_error(void);
 

@@ -15,5 +15,7 @@ from ._abi import (  # noqa: F401
     wal_pq2_matrix, wal_pq2_bytes, wal_pq2_pack, wal_pq2_workspace_bytes, wal_pq2_gemm,
     wal_pq2_body_workspace_bytes, wal_pq2_body_pass,
     wal_base3_bytes, wal_base3_pack, wal_base3_convert,
+    wal_rc1_matrix, wal_rc1_sizes, wal_rc1_prepare, wal_rc1_workspace_bytes, wal_rc1_gemm,
+    wal_rc1_body_workspace_bytes, wal_rc1_body_pass,
 )
-from .packed import PackedMatrix, Pq2Matrix, pack_host, pack_pq2_host, to_device, BodyPass  # noqa: F401
+from .packed import PackedMatrix, Pq2Matrix, Rc1Matrix, pack_host, pack_pq2_host, to_device, BodyPass  # noqa: F401

@@ -28,6 +28,8 @@ EXPORTED_SYMBOLS = [
     "wal_pq2_bytes", "wal_pq2_pack", "wal_pq2_workspace_bytes", "wal_pq2_gemm",
     "wal_pq2_body_workspace_bytes", "wal_pq2_body_pass",
     "wal_base3_bytes", "wal_base3_pack", "wal_base3_convert",
+    "wal_rc1_sizes", "wal_rc1_prepare", "wal_rc1_workspace_bytes", "wal_rc1_gemm",
+    "wal_rc1_body_workspace_bytes", "wal_rc1_body_pass",
     "wal_status_string", "wal_last_error",
 ]
 
@@ -44,6 +46,10 @@ class wal_matrix(ctypes.Structure):
         ("codes", ctypes.c_void_p), ("sites", ctypes.c_void_p), ("scales", ctypes.c_void_p),
         ("u_bits", ctypes.c_void_p), ("v_bits", ctypes.c_void_p), ("lr_scale", ctypes.c_void_p),
     ]
+
+
+class wal_rc1_matrix(ctypes.Structure):
+    _fields_ = wal_matrix._fields_
 
 
 class wal_pq2_matrix(ctypes.Structure):
@@ -92,6 +98,16 @@ lib.wal_base3_bytes.argtypes = [_i, _i]
 lib.wal_base3_bytes.restype = _sz
 lib.wal_base3_pack.argtypes = [_vp, _i, _i, _vp]
 lib.wal_base3_convert.argtypes = [_vp, _vp, _i, _i, _vp, _vp, _vp, _sz, _vp]
+_RP = ctypes.POINTER(wal_rc1_matrix)
+lib.wal_rc1_sizes.argtypes = [_i, _i, _i, _i, _i, ctypes.POINTER(_sz), ctypes.POINTER(_sz)]
+lib.wal_rc1_prepare.argtypes = [_i, _i, _i, _vp, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.wal_rc1_workspace_bytes.argtypes = [_RP, _i]
+lib.wal_rc1_workspace_bytes.restype = _sz
+lib.wal_rc1_gemm.argtypes = [_RP, _vp, _i, _i, _vp, _i, _vp, _sz, _vp]
+lib.wal_rc1_body_workspace_bytes.argtypes = [_RP, _i, _i]
+lib.wal_rc1_body_workspace_bytes.restype = _sz
+lib.wal_rc1_body_pass.argtypes = [ctypes.POINTER(_vp), _RP, _i, ctypes.POINTER(ctypes.c_int32),
+                                  ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp, _sz, _vp]
 lib.wal_status_string.argtypes = [_i]
 lib.wal_status_string.restype = ctypes.c_char_p
 lib.wal_last_error.argtypes = []
@@ -217,3 +233,38 @@ def wal_base3_pack(T, N, K, out):
 def wal_base3_convert(b3, scales_bf16, N, K, codes, alpha, ws, ws_bytes, stream):
     return _check(lib.wal_base3_convert(b3, scales_bf16, N, K, codes, alpha, ws, ws_bytes, stream),
                   "wal_base3_convert")
+
+
+def wal_rc1_sizes(N, K, k, r1, r2):
+    can, prep = (_sz * 7)(), (_sz * 4)()
+    _check(lib.wal_rc1_sizes(N, K, k, r1, r2, can, prep), "wal_rc1_sizes")
+    return [int(v) for v in can], [int(v) for v in prep]
+
+
+def wal_rc1_prepare(N, K, k, scales24, r1, u1, v1, s1, r2, u2, v2, s2, scales32, u_bits, v_bits, lr32, stream):
+    return _check(lib.wal_rc1_prepare(N, K, k, scales24, r1, u1, v1, s1, r2, u2, v2, s2, scales32, u_bits, v_bits,
+                                      lr32, stream), "wal_rc1_prepare")
+
+
+def wal_rc1_workspace_bytes(m, M):
+    return int(lib.wal_rc1_workspace_bytes(ctypes.byref(m), M))
+
+
+def wal_rc1_gemm(m, X, M, ldx, Y, ldy, ws, ws_bytes, stream):
+    return _check(lib.wal_rc1_gemm(ctypes.byref(m), X, M, ldx, Y, ldy, ws, ws_bytes, stream), "wal_rc1_gemm")
+
+
+def wal_rc1_body_workspace_bytes(mats, M):
+    arr = (wal_rc1_matrix * len(mats))(*mats)
+    return int(lib.wal_rc1_body_workspace_bytes(arr, len(mats), M))
+
+
+def wal_rc1_body_pass(plan, mats, stage_of, xs, ys, M, ws, ws_bytes, stream):
+    """plan: a ctypes.c_void_p holding the plan handle (None on the first call)."""
+    n = len(mats)
+    marr = (wal_rc1_matrix * n)(*mats)
+    sarr = (ctypes.c_int32 * n)(*stage_of)
+    xarr = (_vp * n)(*xs)
+    yarr = (_vp * n)(*ys)
+    return _check(lib.wal_rc1_body_pass(ctypes.byref(plan), marr, n, sarr, xarr, yarr, M, ws, ws_bytes,
+                                        stream), "wal_rc1_body_pass")

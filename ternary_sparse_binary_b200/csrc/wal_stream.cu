@@ -72,7 +72,7 @@ constexpr uint32_t kBarrierSpin = 1u << 22;  // polls of the grid-barrier counte
 // (K <= 4096) the rows are contiguous in every buffer and arrive as one copy
 // per buffer, packed at the buffers' own row pitch; otherwise each row is
 // copied on its own at the fixed pitches below.
-constexpr uint32_t kCodePitch = 1024, kSitePitch = 272, kScalePitch = 144;
+constexpr uint32_t kCodePitch = 1024, kSitePitch = 272, kScalePitch = 144, kScalePitch32 = 272;
 // PQ2_0 rows (34-byte blocks: FP16 scale, then 32 code bytes) arrive as one
 // byte range per chunk (one K-slice) or per row (several K-slices, at this
 // pitch: 32 blocks plus the 16-byte widening at both ends).
@@ -80,18 +80,20 @@ constexpr uint32_t kPq2Block = 34, kPq2Pitch = 1152;
 struct ChunkGeom {
   int rpc;                        // rows per chunk
   uint32_t sites, scales, bytes;  // offsets of the site and scale parts, chunk size
+  uint32_t spitch;                // per-row pitch of the scale part (several K-slices)
 };
 __host__ __device__ inline ChunkGeom chunk_geom(int rpc, int fmt) {
   ChunkGeom c;
   c.rpc = rpc;
   if (fmt == kFmtPq2) {
-    c.sites = c.scales = 0u;
+    c.sites = c.scales = c.spitch = 0u;
     c.bytes = (uint32_t)rpc * kPq2Pitch;
     return c;
   }
+  c.spitch = fmt == kFmtF32 ? kScalePitch32 : kScalePitch;  // 32 groups x (8 | 4) bytes + 16
   c.sites = (uint32_t)rpc * kCodePitch;
   c.scales = c.sites + (uint32_t)rpc * kSitePitch;
-  c.bytes = c.scales + (uint32_t)rpc * kScalePitch;
+  c.bytes = c.scales + (uint32_t)rpc * c.spitch;
   return c;
 }
 
@@ -248,7 +250,11 @@ __host__ __device__ inline TileRec tile_record(const GroupDesc& g, const StreamI
 }
 
 __device__ __forceinline__ uint32_t site_bytes(int k) { return (uint32_t)k; }
-__device__ __forceinline__ uint32_t scale_bytes(int k) { return k > 0 ? 4u : 2u; }
+// bytes of one (row, group) in the scale plane: {alpha, beta} or alpha, FP16 or FP32
+template <int FMT>
+__device__ __forceinline__ uint32_t scale_bytes(int k) {
+  return (k > 0 ? 4u : 2u) * (FMT == kFmtF32 ? 2u : 1u);
+}
 
 // Byte range of PQ2_0 blocks [b0, b0 + nb) widened to 16-byte boundaries
 // (the block buffer is zero-padded to a multiple of 16 bytes, so the widened
@@ -291,7 +297,7 @@ __device__ __forceinline__ void issue_chunk(const WarpRing& W, uint32_t sl, uint
     }
     return;
   }
-  const uint32_t kb = site_bytes(W.k), sb = scale_bytes(W.k);
+  const uint32_t kb = site_bytes(W.k), sb = scale_bytes<FMT>(W.k);
   const unsigned char* cbase = reinterpret_cast<const unsigned char*>(W.codes);
   const unsigned char* abase = reinterpret_cast<const unsigned char*>(W.scales);
   if (W.one_slice()) {
@@ -332,7 +338,7 @@ __device__ __forceinline__ void issue_chunk(const WarpRing& W, uint32_t sl, uint
     scale_range(gb, a2, e2);
     bulk_g2s(sl + (uint32_t)u * kCodePitch, cbase + n * (size_t)(W.K / 4) + (size_t)W.s * 1024, (uint32_t)ng * 32u, bar);
     if (e > a) bulk_g2s(sl + C.sites + (uint32_t)u * kSitePitch, W.sites + a, (uint32_t)(e - a), bar);
-    bulk_g2s(sl + C.scales + (uint32_t)u * kScalePitch, abase + a2, (uint32_t)(e2 - a2), bar);
+    bulk_g2s(sl + C.scales + (uint32_t)u * C.spitch, abase + a2, (uint32_t)(e2 - a2), bar);
   }
 }
 
@@ -397,7 +403,7 @@ __device__ __forceinline__ int32_t site_at(uint32_t tab, uint32_t byte) {
 // bytes and scale words for lane 0 of the warp.  `hsw` swaps the two 16-byte
 // halves of the lane's code chunk (matching the limb registers), so that the
 // 32-byte-strided reads of a warp never share a bank.
-template <int KS, bool SIGNED_TABLE>
+template <int KS, bool SIGNED_TABLE, int FMT>
 __device__ __forceinline__ float row_value(uint32_t crow, uint32_t srow, uint32_t arow, int lane, uint32_t hsw,
                                            const uint32_t (&lb)[8][kLimbWords], int32_t xs, float gsc,
                                            uint32_t tab) {
@@ -420,6 +426,11 @@ __device__ __forceinline__ float row_value(uint32_t crow, uint32_t srow, uint32_
   } else if (KS == 2) {
     const uint32_t sw = lds16(srow + (uint32_t)lane * 2u);
     q = site_at<SIGNED_TABLE>(tab, sw & 0xFFu) + site_at<SIGNED_TABLE>(tab, sw >> 8);
+  }
+  if (FMT == kFmtF32) {  // FP32 scales
+    if (KS == 0) return __uint_as_float(ptx::lds32(arow + (uint32_t)lane * 4u)) * ((float)tdot * gsc);
+    const uint2 sc = ptx::lds64(arow + (uint32_t)lane * 8u);
+    return fmaf(__uint_as_float(sc.x), (float)tdot, __uint_as_float(sc.y) * (float)q) * gsc;
   }
   if (KS == 0) {
     const float alpha = fp16_bits_to_float(lds16(arow + (uint32_t)lane * 2u));
@@ -467,18 +478,18 @@ struct RingCtx {
 // Consume this warp's rows of the current group (ring positions q, q+1, ...);
 // after each chunk lane 0 refills the slot with the producer's next chunk.
 // False when a wait gave up.
-template <int KS, bool SIGNED_TABLE>
+template <int KS, bool SIGNED_TABLE, int FMT>
 __device__ __forceinline__ bool run_rows(const WarpRing& W, const RingCtx& R, uint32_t& st, uint32_t& parity, int RB,
                                          int lane, bool active, uint32_t hsw, const uint32_t (&lb)[8][kLimbWords],
                                          int32_t xs, float gsc, uint32_t tab, float* part) {
   const ChunkGeom& C = R.C;
   const int nc = (W.nmine + C.rpc - 1) / C.rpc;
   float* mine = part + W.s * RB + W.r0;  // this warp's row i at mine[i]
-  const uint32_t kb = site_bytes(KS), sb = scale_bytes(KS);
+  const uint32_t kb = site_bytes(KS), sb = scale_bytes<FMT>(KS);
   const bool one = W.one_slice();
   const uint32_t G = (uint32_t)W.G;
   // one slice: pitches of the packed rows; otherwise the fixed pitches
-  const uint32_t cp = one ? G * 32u : kCodePitch, sp = one ? G * kb : kSitePitch, ap = one ? G * sb : kScalePitch;
+  const uint32_t cp = one ? G * 32u : kCodePitch, sp = one ? G * kb : kSitePitch, ap = one ? G * sb : C.spitch;
 #pragma unroll 1
   for (int j = 0; j < nc; ++j) {
     const uint32_t sl = R.ring + st * C.bytes;
@@ -493,7 +504,7 @@ __device__ __forceinline__ bool run_rows(const WarpRing& W, const RingCtx& R, ui
         const uint32_t srow = sl + C.sites + (uint32_t)u * sp + ((gb * kb) & 15u);
         const uint32_t arow = sl + C.scales + (uint32_t)u * ap + ((gb * sb) & 15u);
         const float v =
-            row_value<KS, SIGNED_TABLE>(sl + (uint32_t)u * cp, srow, arow, lane, hsw, lb, xs, gsc, tab);
+            row_value<KS, SIGNED_TABLE, FMT>(sl + (uint32_t)u * cp, srow, arow, lane, hsw, lb, xs, gsc, tab);
         const float tot = warp_sum(active ? v : 0.f);  // fixed butterfly order: reproducible
         if (lane == 0) mine[i] = tot;
       }
@@ -501,7 +512,7 @@ __device__ __forceinline__ bool run_rows(const WarpRing& W, const RingCtx& R, ui
     __syncwarp();  // every lane has consumed the slot before it is refilled
     if (lane == 0) {
       ++R.ps->consumed;
-      prod_topup<kFmtV1>(*R.ps, R.ring, R.mbar, R.stages, R.sched, R.n_groups, R.items, R.warp, C, -1);
+      prod_topup<FMT>(*R.ps, R.ring, R.mbar, R.stages, R.sched, R.n_groups, R.items, R.warp, C, -1);
     }
     if (++st == (uint32_t)R.stages) {
       st = 0;
@@ -733,10 +744,10 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
     if (worker) ok = run_rows_pq2(W, R, st, parity, RB, lane, active, lb, xs, gsc, part);
   } else if (worker) {
     switch (ks) {
-      case 8: ok = run_rows<8, SIGNED_TABLE>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
-      case 4: ok = run_rows<4, SIGNED_TABLE>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
-      case 2: ok = run_rows<2, SIGNED_TABLE>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
-      default: ok = run_rows<0, SIGNED_TABLE>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
+      case 8: ok = run_rows<8, SIGNED_TABLE, FMT>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
+      case 4: ok = run_rows<4, SIGNED_TABLE, FMT>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
+      case 2: ok = run_rows<2, SIGNED_TABLE, FMT>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
+      default: ok = run_rows<0, SIGNED_TABLE, FMT>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
     }
   }
 
@@ -757,7 +768,8 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
   if (tid < r) {
     float a = 0.f;
     for (int s2 = 0; s2 < S; ++s2) a += partz[s2 * WAL_MAX_RANK + tid];
-    s_z[tid] = fp16_bits_to_float(it.lr[tid]) * a;
+    const float s = FMT == kFmtF32 ? reinterpret_cast<const float*>(it.lr)[tid] : fp16_bits_to_float(it.lr[tid]);
+    s_z[tid] = s * a;
   }
   __syncthreads();
   for (int rl = tid; rl < rows; rl += threads) {
@@ -856,8 +868,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
     if (t.rows == 0 || dead) continue;  // uniform across the CTA
     bool ok;
     if (FMT == kFmtPq2) ok = do_group<kFmtPq2, false>(t, R, j, st, parity, area, s_z);
-    else ok = t.signed_table ? do_group<kFmtV1, true>(t, R, j, st, parity, area, s_z)
-                             : do_group<kFmtV1, false>(t, R, j, st, parity, area, s_z);
+    else ok = t.signed_table ? do_group<FMT, true>(t, R, j, st, parity, area, s_z)
+                             : do_group<FMT, false>(t, R, j, st, parity, area, s_z);
     dead = !ok;
   }
   // never leave with bulk copies in flight: after a wait gave up, wait
@@ -893,6 +905,8 @@ int stream_init() {
       e = cudaFuncSetAttribute(stream_kernel<kFmtV1>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_max_smem - 1024);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(stream_kernel<kFmtPq2>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_max_smem - 1024);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(stream_kernel<kFmtF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_max_smem - 1024);
     g_err = e;
   });
   if (g_err != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("device initialisation: ") + cudaGetErrorString(g_err));
@@ -963,7 +977,7 @@ int plan_launch(GroupDesc* groups, int n_groups, bool persistent, int fmt, Strea
     if (!fits) continue;
     for (int j = 0; j < n_groups; ++j) {
       const GroupDesc& g = groups[j];
-      groups[j].signed_table = fmt == kFmtV1 && off + area_plan(g.K, g.S, g.RB, true, fmt).total <= limit ? 1 : 0;
+      groups[j].signed_table = fmt != kFmtPq2 && off + area_plan(g.K, g.S, g.RB, true, fmt).total <= limit ? 1 : 0;
     }
     L.stages = stages;
     L.rpc = rpc;
@@ -998,8 +1012,9 @@ static int launch(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream,
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = cooperative ? 1 : 0;
-  const cudaError_t e = prm.fmt == kFmtPq2 ? cudaLaunchKernelEx(&cfg, stream_kernel<kFmtPq2>, prm)
-                                            : cudaLaunchKernelEx(&cfg, stream_kernel<kFmtV1>, prm);
+  const cudaError_t e = prm.fmt == kFmtPq2   ? cudaLaunchKernelEx(&cfg, stream_kernel<kFmtPq2>, prm)
+                        : prm.fmt == kFmtF32 ? cudaLaunchKernelEx(&cfg, stream_kernel<kFmtF32>, prm)
+                                             : cudaLaunchKernelEx(&cfg, stream_kernel<kFmtV1>, prm);
   if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("stream_kernel launch: ") + cudaGetErrorString(e));
   return WAL_OK;
 }
@@ -1015,9 +1030,10 @@ int launch_stream(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream)
 int launch_body(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream) {
   if (!prm.t_sched || !prm.t_items || !prm.barrier) return fail(WAL_ERR_ARG, "body launch without tables");
   int per_sm = 0;
-  cudaError_t e = prm.fmt == kFmtPq2
-                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, stream_kernel<kFmtPq2>, L.threads, L.smem)
-                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, stream_kernel<kFmtV1>, L.threads, L.smem);
+  const void* fn = prm.fmt == kFmtPq2   ? reinterpret_cast<const void*>(stream_kernel<kFmtPq2>)
+                   : prm.fmt == kFmtF32 ? reinterpret_cast<const void*>(stream_kernel<kFmtF32>)
+                                        : reinterpret_cast<const void*>(stream_kernel<kFmtV1>);
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, L.threads, L.smem);
   if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("occupancy query: ") + cudaGetErrorString(e));
   if (per_sm < 1 || L.grid > per_sm * num_sms())
     return fail(WAL_ERR_UNSUPPORTED, "the persistent launch does not fit on the device at once");

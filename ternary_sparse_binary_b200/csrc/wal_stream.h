@@ -12,8 +12,11 @@ constexpr int kMaxItems = 16;
 // Weight formats a launch can stream (one per launch):
 //  kFmtV1  layout v1 of the direct-packed product (codes, sites, scales, WALB2);
 //  kFmtPq2 PQ2_0 plain-ternary blocks (FP16 scale + 32 code bytes per 128
-//          weights); `codes` then points at the block buffer, k = r = 0.
-enum : int { kFmtV1 = 0, kFmtPq2 = 1 };
+//          weights); `codes` then points at the block buffer, k = r = 0;
+//  kFmtF32 layout v1 with FP32 scales: {alpha, beta} as two floats per
+//          (row, group) (alpha alone when k = 0) and FP32 per-rank scales (a
+//          prepared RC1 matrix); `scales` and `lr` then point at floats.
+enum : int { kFmtV1 = 0, kFmtPq2 = 1, kFmtF32 = 2 };
 
 // One product y = W x.
 struct StreamItem {
@@ -64,7 +67,7 @@ struct StreamParams {
   uint32_t area_off;          // shared-memory offset of the per-group area
   unsigned int* barrier;      // grid-barrier counter (zeroed before the launch), body pass only
   int32_t* status;            // workspace status word (may be NULL)
-  int fmt;                    // kFmtV1 or kFmtPq2
+  int fmt;                    // kFmtV1, kFmtPq2 or kFmtF32
 };
 
 struct StreamLaunch {

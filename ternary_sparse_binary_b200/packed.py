@@ -5,7 +5,7 @@ import numpy as np
 import torch
 
 from . import _abi
-from ._abi import wal_matrix, wal_pq2_matrix
+from ._abi import wal_matrix, wal_pq2_matrix, wal_rc1_matrix
 
 
 def _ptr(a):
@@ -78,6 +78,47 @@ class Pq2Matrix:
         return _abi.wal_pq2_workspace_bytes(self.desc, M)
 
 
+def _dev(a, device):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.uint8).reshape(-1)).to(device)
+
+
+class Rc1Matrix:
+    """A prepared RC1 matrix on a CUDA device: the layout-v1 code plane and
+    site bytes, FP32 scales and one WALB2 rank block, with its
+    wal_rc1_matrix descriptor.  Built by prepare() from the canonical planes
+    (24-bit scales, two paths) with the library's GPU prepare step."""
+
+    def __init__(self, N, K, k, r, codes, sites, scales32, u_bits, v_bits, lr32):
+        self.N, self.K, self.k, self.r = N, K, k, r
+        self.bufs = [codes, sites, scales32, u_bits, v_bits, lr32]
+        ptr = lambda t: t.data_ptr() if t is not None and t.numel() else None
+        self.desc = wal_rc1_matrix(N, K, k, r, *[ptr(b) for b in self.bufs])
+
+    @classmethod
+    def prepare(cls, codes, sites, scales24, path1, path2, N, K, k, device="cuda", stream=None):
+        """codes, sites: layout-v1 host planes; scales24: host bytes of the
+        24-bit scale plane; path1, path2: (r_p, u_bits, v_bits, s24) host
+        planes (r_p may be 0 with None buffers)."""
+        (r1, u1, v1, s1), (r2, u2, v2, s2) = path1, path2
+        _, prep = _abi.wal_rc1_sizes(N, K, k, r1, r2)
+        d = lambda a: _dev(a, device) if a is not None and np.size(a) else None
+        c, st, s24 = d(codes), d(sites), d(scales24)
+        ins = [d(u1), d(v1), d(s1), d(u2), d(v2), d(s2)]
+        out = [torch.zeros(n, dtype=torch.uint8, device=device) if n else None for n in prep]
+        ptr = lambda t: t.data_ptr() if t is not None else None
+        _abi.wal_rc1_prepare(N, K, k, ptr(s24), r1, ptr(ins[0]), ptr(ins[1]), ptr(ins[2]), r2, ptr(ins[3]),
+                             ptr(ins[4]), ptr(ins[5]), *[ptr(o) for o in out], _stream_handle(stream))
+        torch.cuda.current_stream(device).synchronize() if stream is None else stream.synchronize()
+        return cls(N, K, k, r1 + r2, c, st, *out)
+
+    @property
+    def nbytes(self):
+        return sum(b.numel() for b in self.bufs if b is not None)
+
+    def workspace_bytes(self, M=1):
+        return _abi.wal_rc1_workspace_bytes(self.desc, M)
+
+
 def to_device(bufs, N, K, k, r, device="cuda"):
     return PackedMatrix(bufs, N, K, k, r, device)
 
@@ -89,24 +130,30 @@ def _stream_handle(stream=None):
 
 class BodyPass:
     """Owns a wal_body_plan handle and its workspace; run() replays the graph.
-    The matrices are all PackedMatrix (layout v1) or all Pq2Matrix (PQ2_0)."""
+    The matrices are all PackedMatrix (layout v1), all Pq2Matrix (PQ2_0) or
+    all Rc1Matrix (prepared RC1)."""
 
     def __init__(self, mats, stage_of, xs, ys, M=1, device="cuda"):
         self.mats = list(mats)
         self.descs = [m.desc for m in self.mats]
-        self.pq2 = isinstance(self.mats[0], Pq2Matrix)
-        if any(isinstance(m, Pq2Matrix) != self.pq2 for m in self.mats):
+        kind = type(self.mats[0])
+        if any(type(m) is not kind for m in self.mats):
             raise ValueError("a body pass takes matrices of one format")
+        self._ws_fn, self._pass_fn = {
+            PackedMatrix: (_abi.wal_body_workspace_bytes, _abi.wal_body_pass),
+            Pq2Matrix: (_abi.wal_pq2_body_workspace_bytes, _abi.wal_pq2_body_pass),
+            Rc1Matrix: (_abi.wal_rc1_body_workspace_bytes, _abi.wal_rc1_body_pass),
+        }[kind]
         self.stage_of = [int(s) for s in stage_of]
         self.xs, self.ys, self.M = list(xs), list(ys), M
-        nb = (_abi.wal_pq2_body_workspace_bytes if self.pq2 else _abi.wal_body_workspace_bytes)(self.descs, M)
+        nb = self._ws_fn(self.descs, M)
         if nb == 0:
             raise _abi.WalError(_abi.WAL_ERR_ARG, "wal_body_workspace_bytes")
         self.ws = torch.empty(nb, dtype=torch.uint8, device=device)
         self.plan = ctypes.c_void_p(None)
 
     def run(self, stream=None):
-        (_abi.wal_pq2_body_pass if self.pq2 else _abi.wal_body_pass)(self.plan, self.descs, self.stage_of, [x.data_ptr() for x in self.xs],
+        self._pass_fn(self.plan, self.descs, self.stage_of, [x.data_ptr() for x in self.xs],
                            [y.data_ptr() for y in self.ys], self.M, self.ws.data_ptr(), self.ws.numel(),
                            _stream_handle(stream))
 

@@ -30,5 +30,6 @@ from .gen import (  # noqa: F401
     CONFIG_SEED,
     LAYER_8B,
     LAYER_27B,
+    ROLE_K_27B,
     stream_seed,
 )
