@@ -24,6 +24,8 @@ from .gen import (  # noqa: F401
     gen_pq2,
     gen_base3,
     gen_rc1,
+    gen_int4,
+    gen_int3,
     f24_bytes_from_f32,
     workload_id,
     WORKLOAD_IDS,

@@ -283,3 +283,23 @@ def gen_rc1(N: int, K: int, k: int, r1: int, r2: int, config_id: int = 0, matrix
         paths += [U, V, s]
     return dict(N=N, K=K, k=k, T=c.T, site_pos=c.site_pos, site_sign=c.site_sign, alpha24=alpha, beta24=beta,
                 U1=paths[0], V1=paths[1], s1=paths[2], U2=paths[3], V2=paths[4], s2=paths[5])
+
+
+def gen_int4(N: int, K: int, config_id: int = 0, matrix_index: int = 0):
+    """An INT4/g128 matrix (the LM head): q iid uniform on [-8, 7] and one
+    scale d = fp16(|N(0, 0.02)|) per (row, 128-group).  Returns (q int8 [N, K],
+    d uint16 fp16 bits [N, K/128])."""
+    rq = rng_for(config_id, matrix_index, S_T)
+    q = rq.integers(-8, 8, size=(N, K), dtype=np.int8)
+    rs = rng_for(config_id, matrix_index, S_SCALES)
+    return q, _fp16_bits(np.abs(rs.normal(0.0, 0.02, size=(N, K // GROUP))))
+
+
+def gen_int3(V: int, H: int, config_id: int = 0, matrix_index: int = 0):
+    """An INT3/g128 table (the embedding): q iid uniform on [-4, 3] and one
+    scale d = fp16(|N(0, 0.02)|) per (row, 128-group).  Returns (q int8 [V, H],
+    d uint16 fp16 bits [V, H/128])."""
+    rq = rng_for(config_id, matrix_index, S_T)
+    q = rq.integers(-4, 4, size=(V, H), dtype=np.int8)
+    rs = rng_for(config_id, matrix_index, S_SCALES)
+    return q, _fp16_bits(np.abs(rs.normal(0.0, 0.02, size=(V, H // GROUP))))
