@@ -150,7 +150,8 @@ int wal_gemm_tc_noalloc(const wal_matrix* m, const uint16_t* X, int M, int ldx, 
 
 /* Read and clear the device status word in a workspace header (synchronises
  * `stream`).  Every product call clears the word when it starts, so it reports
- * on the last call that used this workspace.  WAL_OK or WAL_ERR_TIMEOUT. */
+ * on the last call that used this workspace.  WAL_OK, WAL_ERR_TIMEOUT, or
+ * WAL_ERR_ARG for a token id outside the table (wal_int3_embed). */
 int wal_device_status(void* ws, wal_stream_t stream);
 
 /* Whole body pass: n_mats products, matrix i reading xs[i] (bf16 [M][K_i]) and
@@ -301,6 +302,51 @@ size_t wal_rc1_body_workspace_bytes(const wal_rc1_matrix* mats, int n_mats, int 
 int wal_rc1_body_pass(wal_body_plan** plan, const wal_rc1_matrix* mats, int n_mats, const int32_t* stage_of,
                       const uint16_t* const* xs, float* const* ys, int M, void* ws, size_t ws_bytes,
                       wal_stream_t stream);
+
+/* ---- around the body: INT3/g128 embedding, INT4/g128 LM head --------------
+ * The WAL-Ternary-8B card (Kazakh README, "Model format") keeps the
+ * embedding as INT3 and the LM head as INT4, both with groups of 128.  This
+ * library's reading: w = d * q with an FP16 scale d per (row, 128 columns);
+ * codes are offset binary, u = q + 8 (INT4, q in [-8, 7]) or u = q + 4
+ * (INT3, q in [-4, 3]).  INT4 rows: K / 2 bytes, column 2i in the low nibble
+ * of byte i.  INT3 rows: 48 bytes per group, code j of the group at bits
+ * 3j .. 3j + 2 of its little-endian 384-bit string.  Scales fp16 [rows][K/128].
+ * Every plane is zero-padded to a multiple of 16 bytes. */
+typedef struct wal_int4_matrix {  /* device pointers, 16-byte aligned */
+  int32_t N, K;                   /* K a positive multiple of 128, at most 24576 */
+  const uint8_t* codes;           /* [N][K/2] */
+  const uint16_t* scales;         /* fp16 [N][K/128] */
+} wal_int4_matrix;
+typedef struct wal_int3_table {   /* device pointers, 16-byte aligned */
+  int32_t V, H;                   /* rows (vocabulary) and row length */
+  const uint8_t* codes;           /* [V][H/128][48] */
+  const uint16_t* scales;         /* fp16 [V][H/128] */
+} wal_int3_table;
+
+/* Plane sizes (codes, scales) in bytes.  Host only; WAL_ERR_SHAPE on a bad shape. */
+int wal_int4_sizes(int N, int K, size_t out[2]);
+int wal_int3_sizes(int V, int H, size_t out[2]);
+
+/* Host packers: q int8 [rows][cols], d fp16 bits [rows][cols/128] into the
+ * two planes (host memory of the wal_*_sizes sizes, padding zeroed).
+ * WAL_ERR_FORMAT when a value leaves its range. */
+int wal_int4_pack(const int8_t* q, const uint16_t* d, int N, int K, void* codes, void* scales);
+int wal_int3_pack(const int8_t* q, const uint16_t* d, int V, int H, void* codes, void* scales);
+
+/* LM head: Y[M][ldy] = X[M][ldx] W^T for 1 <= M <= 16 (logits, FP32), with
+ * the contract of wal_gemm_small_m.  Runs the INT4 specialisation of the
+ * decode-GEMV. */
+size_t wal_int4_workspace_bytes(const wal_int4_matrix* m, int M);
+int wal_int4_gemm(const wal_int4_matrix* m, const uint16_t* X, int M, int ldx, float* Y, int ldy, void* ws,
+                  size_t ws_bytes, wal_stream_t stream);
+
+/* Embedding gather: out[m][0..H) = d[ids[m]] * q[ids[m]] in FP32 (exact),
+ * for M >= 1 token ids (int32, device memory).  out is device memory [M][H],
+ * 16-byte aligned.  An id outside [0, V) gives a zero row and records
+ * WAL_ERR_ARG in the workspace status word (wal_device_status); ws: at least
+ * 512 bytes.  Asynchronous. */
+int wal_int3_embed(const wal_int3_table* t, const int32_t* ids, int M, float* out, void* ws, size_t ws_bytes,
+                   wal_stream_t stream);
 
 const char* wal_status_string(int status);
 const char* wal_last_error(void);

@@ -17,5 +17,7 @@ from ._abi import (  # noqa: F401
     wal_base3_bytes, wal_base3_pack, wal_base3_convert,
     wal_rc1_matrix, wal_rc1_sizes, wal_rc1_prepare, wal_rc1_workspace_bytes, wal_rc1_gemm,
     wal_rc1_body_workspace_bytes, wal_rc1_body_pass,
+    wal_int4_matrix, wal_int3_table, wal_int4_sizes, wal_int3_sizes, wal_int4_pack, wal_int3_pack,
+    wal_int4_workspace_bytes, wal_int4_gemm, wal_int3_embed,
 )
 from .packed import PackedMatrix, Pq2Matrix, Rc1Matrix, pack_host, pack_pq2_host, to_device, BodyPass  # noqa: F401

@@ -30,6 +30,8 @@ EXPORTED_SYMBOLS = [
     "wal_base3_bytes", "wal_base3_pack", "wal_base3_convert",
     "wal_rc1_sizes", "wal_rc1_prepare", "wal_rc1_workspace_bytes", "wal_rc1_gemm",
     "wal_rc1_body_workspace_bytes", "wal_rc1_body_pass",
+    "wal_int4_sizes", "wal_int3_sizes", "wal_int4_pack", "wal_int3_pack", "wal_int4_workspace_bytes",
+    "wal_int4_gemm", "wal_int3_embed",
     "wal_status_string", "wal_last_error",
 ]
 
@@ -50,6 +52,14 @@ class wal_matrix(ctypes.Structure):
 
 class wal_rc1_matrix(ctypes.Structure):
     _fields_ = wal_matrix._fields_
+
+
+class wal_int4_matrix(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class wal_int3_table(ctypes.Structure):
+    _fields_ = [("V", ctypes.c_int32), ("H", ctypes.c_int32), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
 
 
 class wal_pq2_matrix(ctypes.Structure):
@@ -108,6 +118,14 @@ lib.wal_rc1_body_workspace_bytes.argtypes = [_RP, _i, _i]
 lib.wal_rc1_body_workspace_bytes.restype = _sz
 lib.wal_rc1_body_pass.argtypes = [ctypes.POINTER(_vp), _RP, _i, ctypes.POINTER(ctypes.c_int32),
                                   ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp, _sz, _vp]
+lib.wal_int4_sizes.argtypes = [_i, _i, ctypes.POINTER(_sz)]
+lib.wal_int3_sizes.argtypes = [_i, _i, ctypes.POINTER(_sz)]
+lib.wal_int4_pack.argtypes = [_vp, _vp, _i, _i, _vp, _vp]
+lib.wal_int3_pack.argtypes = [_vp, _vp, _i, _i, _vp, _vp]
+lib.wal_int4_workspace_bytes.argtypes = [ctypes.POINTER(wal_int4_matrix), _i]
+lib.wal_int4_workspace_bytes.restype = _sz
+lib.wal_int4_gemm.argtypes = [ctypes.POINTER(wal_int4_matrix), _vp, _i, _i, _vp, _i, _vp, _sz, _vp]
+lib.wal_int3_embed.argtypes = [ctypes.POINTER(wal_int3_table), _vp, _i, _vp, _vp, _sz, _vp]
 lib.wal_status_string.argtypes = [_i]
 lib.wal_status_string.restype = ctypes.c_char_p
 lib.wal_last_error.argtypes = []
@@ -268,3 +286,35 @@ def wal_rc1_body_pass(plan, mats, stage_of, xs, ys, M, ws, ws_bytes, stream):
     yarr = (_vp * n)(*ys)
     return _check(lib.wal_rc1_body_pass(ctypes.byref(plan), marr, n, sarr, xarr, yarr, M, ws, ws_bytes,
                                         stream), "wal_rc1_body_pass")
+
+
+def wal_int4_sizes(N, K):
+    out = (_sz * 2)()
+    _check(lib.wal_int4_sizes(N, K, out), "wal_int4_sizes")
+    return [int(v) for v in out]
+
+
+def wal_int3_sizes(V, H):
+    out = (_sz * 2)()
+    _check(lib.wal_int3_sizes(V, H, out), "wal_int3_sizes")
+    return [int(v) for v in out]
+
+
+def wal_int4_pack(q, d, N, K, codes, scales):
+    return _check(lib.wal_int4_pack(q, d, N, K, codes, scales), "wal_int4_pack")
+
+
+def wal_int3_pack(q, d, V, H, codes, scales):
+    return _check(lib.wal_int3_pack(q, d, V, H, codes, scales), "wal_int3_pack")
+
+
+def wal_int4_workspace_bytes(m, M):
+    return int(lib.wal_int4_workspace_bytes(ctypes.byref(m), M))
+
+
+def wal_int4_gemm(m, X, M, ldx, Y, ldy, ws, ws_bytes, stream):
+    return _check(lib.wal_int4_gemm(ctypes.byref(m), X, M, ldx, Y, ldy, ws, ws_bytes, stream), "wal_int4_gemm")
+
+
+def wal_int3_embed(t, ids, M, out, ws, ws_bytes, stream):
+    return _check(lib.wal_int3_embed(ctypes.byref(t), ids, M, out, ws, ws_bytes, stream), "wal_int3_embed")

@@ -6,7 +6,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libwal.so")
-SOURCES = ["wal_host.cpp", "wal_gemv.cu", "wal_stream.cu", "wal_body.cu", "wal_tc.cu", "wal_noalloc.cu", "wal_pq2.cu", "wal_base3.cu", "wal_rc1.cu"]
+SOURCES = ["wal_host.cpp", "wal_gemv.cu", "wal_stream.cu", "wal_body.cu", "wal_tc.cu", "wal_noalloc.cu", "wal_pq2.cu", "wal_base3.cu", "wal_rc1.cu", "wal_head.cu"]
 HEADERS = ["wal_internal.h", "wal_device.cuh", "wal_stream.h", "wal_ptx.cuh", "wal_tc.h", os.path.join("..", "..", "include", "wal.h")]
 
 NVCC_FLAGS = [

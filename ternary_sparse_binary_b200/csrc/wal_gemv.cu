@@ -267,6 +267,7 @@ extern "C" int wal_device_status(void* ws, wal_stream_t stream) {
   if (e == cudaSuccess) e = cudaMemsetAsync(word, 0, 4, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "device status readback");
+  if (h == WAL_ERR_ARG) return fail(WAL_ERR_ARG, "a token id is outside the embedding table");
   if (h != 0) return fail(WAL_ERR_TIMEOUT, "a bounded device wait gave up");
   return WAL_OK;
 }

@@ -82,9 +82,17 @@ struct ChunkGeom {
   uint32_t sites, scales, bytes;  // offsets of the site and scale parts, chunk size
   uint32_t spitch;                // per-row pitch of the scale part (several K-slices)
 };
+// Code bytes of one 128-group: 2-bit codes, or 4-bit INT4 codes.
+__host__ __device__ constexpr uint32_t code_group_bytes(int fmt) { return fmt == kFmtInt4 ? 64u : 32u; }
 __host__ __device__ inline ChunkGeom chunk_geom(int rpc, int fmt) {
   ChunkGeom c;
   c.rpc = rpc;
+  if (fmt == kFmtInt4) {  // codes (32 groups x 64 B per row), no sites, fp16 scales
+    c.spitch = kScalePitch;
+    c.sites = c.scales = (uint32_t)rpc * 32u * code_group_bytes(fmt);
+    c.bytes = c.scales + (uint32_t)rpc * kScalePitch;
+    return c;
+  }
   if (fmt == kFmtPq2) {
     c.sites = c.scales = c.spitch = 0u;
     c.bytes = (uint32_t)rpc * kPq2Pitch;
@@ -163,6 +171,33 @@ __device__ __forceinline__ int32_t group_dot(const uint32_t (&wv)[8], const uint
   return (int32_t)(((uint32_t)t2 << 16) + (t1 << 8) + t0);
 }
 
+// Exact integer sum_j u_j X_j over one lane's INT4 group (16 code words of
+// eight 4-bit codes u = q + 8).  Word i of the group holds columns 8i..8i+7;
+// its low nibbles (word & 0x0F0F0F0F) are the even columns and its high
+// nibbles the odd ones, matched by limb slots 2h and 2h + 1 of 16-column
+// word i / 2 (h = i % 2).  Both slots carry the code itself (no slot
+// weight), so the three limb sums need no fold.  |X| < 2^20 keeps the true
+// sum_j q_j X_j inside int32; the uint32 arithmetic wraps to it.
+__device__ __forceinline__ uint32_t group_dot4(const uint32_t (&wv)[16], const uint32_t (&lb)[8][kLimbWords]) {
+  uint32_t a0 = 0u, a1 = 0u;
+  int32_t a2 = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t word = wv[2 * w + h];
+      const uint32_t lo = word & 0x0F0F0F0Fu, hi = (word >> 4) & 0x0F0F0F0Fu;
+      a0 = dp4a_uu(lo, lb[w][0 * 4 + 2 * h], a0);
+      a0 = dp4a_uu(hi, lb[w][0 * 4 + 2 * h + 1], a0);
+      a1 = dp4a_uu(lo, lb[w][1 * 4 + 2 * h], a1);
+      a1 = dp4a_uu(hi, lb[w][1 * 4 + 2 * h + 1], a1);
+      a2 = dp4a_us(lo, lb[w][2 * 4 + 2 * h], a2);
+      a2 = dp4a_us(hi, lb[w][2 * 4 + 2 * h + 1], a2);
+    }
+  }
+  return a0 + (a1 << 8) + ((uint32_t)a2 << 16);
+}
+
 // ---------------------------------------------------------------------------
 // shared memory: [ring | mbarriers | producer states] then the per-group area
 // ---------------------------------------------------------------------------
@@ -187,7 +222,7 @@ __host__ __device__ inline AreaPlan area_plan(int K, int S, int RB, bool signed_
   uint32_t off = 0;
   auto take = [&](uint32_t bytes) { uint32_t o = off; off = (off + bytes + 15u) & ~15u; return o; };
   const uint32_t G = (uint32_t)K / kGroup;
-  const bool v1 = fmt != kFmtPq2;
+  const bool v1 = fmt == kFmtV1 || fmt == kFmtF32;
   p.table = take(v1 ? G * table_stride(signed_table) * 4u : 0u);
   p.limbs = take(G * kLimbStride * 4u);
   p.part = take((uint32_t)S * RB * 4u);  // one partial per (slice, row)
@@ -300,13 +335,14 @@ __device__ __forceinline__ void issue_chunk(const WarpRing& W, uint32_t sl, uint
   const uint32_t kb = site_bytes(W.k), sb = scale_bytes<FMT>(W.k);
   const unsigned char* cbase = reinterpret_cast<const unsigned char*>(W.codes);
   const unsigned char* abase = reinterpret_cast<const unsigned char*>(W.scales);
+  constexpr uint32_t cgb = code_group_bytes(FMT);  // code bytes per group
   if (W.one_slice()) {
     const size_t n = (size_t)(W.nb + i0), G = (size_t)W.G;
-    const uint32_t clen = (uint32_t)un * (uint32_t)(W.K / 4);
+    const uint32_t clen = (uint32_t)un * (uint32_t)W.G * cgb;
     const size_t sa = (n * G * kb) & ~(size_t)15, se = ((n + un) * G * kb + 15) & ~(size_t)15;
     const size_t aa = (n * G * sb) & ~(size_t)15, ae = ((n + un) * G * sb + 15) & ~(size_t)15;
     mbar_arrive_expect_tx(bar, clen + (uint32_t)(se - sa) + (uint32_t)(ae - aa));
-    bulk_g2s(sl, cbase + n * (size_t)(W.K / 4), clen, bar);
+    bulk_g2s(sl, cbase + n * G * cgb, clen, bar);
     if (se > sa) bulk_g2s(sl + C.sites, W.sites + sa, (uint32_t)(se - sa), bar);
     bulk_g2s(sl + C.scales, abase + aa, (uint32_t)(ae - aa), bar);
     return;
@@ -327,7 +363,7 @@ __device__ __forceinline__ void issue_chunk(const WarpRing& W, uint32_t sl, uint
     size_t a, e, a2, e2;
     site_range(gb, a, e);
     scale_range(gb, a2, e2);
-    bytes += (uint32_t)ng * 32u + (uint32_t)(e - a) + (uint32_t)(e2 - a2);
+    bytes += (uint32_t)ng * cgb + (uint32_t)(e - a) + (uint32_t)(e2 - a2);
   }
   mbar_arrive_expect_tx(bar, bytes);
   for (int u = 0; u < un; ++u) {
@@ -336,7 +372,8 @@ __device__ __forceinline__ void issue_chunk(const WarpRing& W, uint32_t sl, uint
     size_t a, e, a2, e2;
     site_range(gb, a, e);
     scale_range(gb, a2, e2);
-    bulk_g2s(sl + (uint32_t)u * kCodePitch, cbase + n * (size_t)(W.K / 4) + (size_t)W.s * 1024, (uint32_t)ng * 32u, bar);
+    bulk_g2s(sl + (uint32_t)u * 32u * cgb, cbase + n * (size_t)W.G * cgb + (size_t)W.s * 32u * cgb, (uint32_t)ng * cgb,
+             bar);
     if (e > a) bulk_g2s(sl + C.sites + (uint32_t)u * kSitePitch, W.sites + a, (uint32_t)(e - a), bar);
     bulk_g2s(sl + C.scales + (uint32_t)u * C.spitch, abase + a2, (uint32_t)(e2 - a2), bar);
   }
@@ -407,6 +444,20 @@ template <int KS, bool SIGNED_TABLE, int FMT>
 __device__ __forceinline__ float row_value(uint32_t crow, uint32_t srow, uint32_t arow, int lane, uint32_t hsw,
                                            const uint32_t (&lb)[8][kLimbWords], int32_t xs, float gsc,
                                            uint32_t tab) {
+  if (FMT == kFmtInt4) {
+    // the lane's 64 code bytes as four 16-byte reads starting at chunk
+    // (lane / 2) % 4, so that the 8 lanes of each quarter-warp hit 8
+    // different 16-byte bank groups; the limb image is rotated to match
+    const uint32_t cd = crow + (uint32_t)lane * 64u, rot = ((uint32_t)lane >> 1) & 3u;
+    uint32_t wv[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 c = lds128(cd + 16u * (((uint32_t)j + rot) & 3u));
+      wv[4 * j] = c.x; wv[4 * j + 1] = c.y; wv[4 * j + 2] = c.z; wv[4 * j + 3] = c.w;
+    }
+    const int32_t tdot = (int32_t)(group_dot4(wv, lb) - 8u * (uint32_t)xs);
+    return fp16_bits_to_float(lds16(arow + (uint32_t)lane * 2u)) * ((float)tdot * gsc);
+  }
   const uint32_t cd = crow + (uint32_t)lane * 32u;
   const uint4 c0 = lds128(cd + hsw), c1 = lds128(cd + (hsw ^ 16u));
   const uint32_t wv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -489,7 +540,8 @@ __device__ __forceinline__ bool run_rows(const WarpRing& W, const RingCtx& R, ui
   const bool one = W.one_slice();
   const uint32_t G = (uint32_t)W.G;
   // one slice: pitches of the packed rows; otherwise the fixed pitches
-  const uint32_t cp = one ? G * 32u : kCodePitch, sp = one ? G * kb : kSitePitch, ap = one ? G * sb : C.spitch;
+  constexpr uint32_t cgb = code_group_bytes(FMT);
+  const uint32_t cp = one ? G * cgb : 32u * cgb, sp = one ? G * kb : kSitePitch, ap = one ? G * sb : C.spitch;
 #pragma unroll 1
   for (int j = 0; j < nc; ++j) {
     const uint32_t sl = R.ring + st * C.bytes;
@@ -571,11 +623,17 @@ __device__ __forceinline__ void load_x(const uint16_t* x, int K, uint4 (&xr)[kMa
   }
 }
 
-// PQ2 = true: no site table, and the limb image keeps every group in natural
-// word order (PQ2_0 code words are read one by one, not as 16-byte halves).
-template <bool SIGNED_TABLE, bool PQ2>
+// Layout v1 (and its FP32-scale form): the site table and the half-swapped
+// limb image below.  PQ2_0: no site table, and the image keeps every group in
+// natural word order (its code words are read one by one).  INT4: no site
+// table, X scaled to 20 bits (X = round(x * 2^(19 - e_g))), the limb slots of
+// each 16-column word are (8-column half, even / odd column), and a group's
+// words are stored rotated by 2 * ((g / 2) % 4) to match its lane's reads.
+template <bool SIGNED_TABLE, int FMT>
 __device__ __forceinline__ void build_image(const uint4 (&xr)[kMaxXChunks], int K, unsigned char* area,
                                             const AreaPlan& ap) {
+  constexpr bool NO_TABLE = FMT == kFmtPq2 || FMT == kFmtInt4, INT4 = FMT == kFmtInt4;
+  constexpr uint32_t kOff = INT4 ? 19u : 21u;  // X = round(x * 2^(kOff - e_g))
   const int threads = blockDim.x, tid = threadIdx.x, lane = tid & 31;
   const uint32_t tstride = table_stride(SIGNED_TABLE);
   int32_t* table = reinterpret_cast<int32_t*>(area + ap.table);
@@ -602,9 +660,9 @@ __device__ __forceinline__ void build_image(const uint4 (&xr)[kMaxXChunks], int 
     for (int off = 8; off; off >>= 1) mx = max(mx, __shfl_xor_sync(gmask, mx, off));
     uint32_t emax = mx >> 7;
     emax = emax > 1u ? emax : 1u;  // exponent field of the group maximum (denormals as 1)
-    // X = round(x * 2^(148 - emax)); tiny groups are pre-scaled by 2^64 so the factor stays finite
+    // X = round(x * 2^(127 + kOff - emax)); tiny groups are pre-scaled by 2^64 so the factor stays finite
     const float pre = emax < 64u ? 18446744073709551616.0f : 1.0f;
-    const float scl = __uint_as_float((275u - emax - (emax < 64u ? 64u : 0u)) << 23);
+    const float scl = __uint_as_float((254u + kOff - emax - (emax < 64u ? 64u : 0u)) << 23);
     int32_t X[8];
     int32_t sum8 = 0;
 #pragma unroll
@@ -621,20 +679,36 @@ __device__ __forceinline__ void build_image(const uint4 (&xr)[kMaxXChunks], int 
     // A group read by a lane with bit 2 set is stored with its halves swapped
     // (words 0-3 <-> 4-7), the order in which that lane holds its limbs, so
     // that every lane reads its image front to back without bank conflicts.
-    const int wl = ((c >> 4) & 7) ^ ((!PQ2 && (gg & 4)) ? 4 : 0);
-    uint16_t* img16 = reinterpret_cast<uint16_t*>(limbs + (size_t)gg * kLimbStride);
+    if (INT4) {
+      // byte b of (word wl, limb L, slot 2h + p) = limb L of column 16 wl + 8h + 2b + p
+      const int wl = (((c >> 4) & 7) - 2 * ((gg >> 1) & 3)) & 7;
+      uint32_t* img32 = limbs + (size_t)gg * kLimbStride;
 #pragma unroll
-    for (int L2 = 0; L2 < 3; ++L2)
+      for (int L2 = 0; L2 < 3; ++L2)
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        img16[((wl * 3 + L2) * 4 + q) * 2 + h] =
-            (uint16_t)__byte_perm((uint32_t)X[q], (uint32_t)X[4 + q], (uint32_t)(L2 | ((4 + L2) << 4)));
+        for (int p = 0; p < 2; ++p) {
+          const uint32_t sel = (uint32_t)(L2 | ((4 + L2) << 4));
+          const uint32_t b01 = __byte_perm((uint32_t)X[p], (uint32_t)X[2 + p], sel);
+          const uint32_t b23 = __byte_perm((uint32_t)X[4 + p], (uint32_t)X[6 + p], sel);
+          img32[(wl * 3 + L2) * 4 + 2 * h + p] = __byte_perm(b01, b23, 0x5410u);
+        }
+    } else {
+      const int wl = ((c >> 4) & 7) ^ ((!NO_TABLE && (gg & 4)) ? 4 : 0);
+      uint16_t* img16 = reinterpret_cast<uint16_t*>(limbs + (size_t)gg * kLimbStride);
+#pragma unroll
+      for (int L2 = 0; L2 < 3; ++L2)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          img16[((wl * 3 + L2) * 4 + q) * 2 + h] =
+              (uint16_t)__byte_perm((uint32_t)X[q], (uint32_t)X[4 + q], (uint32_t)(L2 | ((4 + L2) << 4)));
+    }
     if ((c8 & 15) == 0) {
       xgsum[gg] = sum8;
-      gsc_s[gg] = emax >= 22u ? __uint_as_float((emax - 21u) << 23) : __uint_as_float(1u << (emax + 1u));
+      // 2^(emax - 127 - kOff), a subnormal float for the smallest exponents
+      gsc_s[gg] = emax > kOff ? __uint_as_float((emax - kOff) << 23) : __uint_as_float(1u << (emax + 22u - kOff));
     }
     // site table: entry e of group gg (e = site byte) at gg * stride + e
-    if (!PQ2) {
+    if (!NO_TABLE) {
       int32_t* trow = table + (size_t)gg * tstride + pos;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
@@ -661,7 +735,8 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
   WarpRing W;
   warp_work(t, &it, warp, W);
   constexpr bool PQ2 = FMT == kFmtPq2;
-  const int r = PQ2 ? 0 : it.r, ks = PQ2 ? 0 : it.k;
+  constexpr bool PLAIN = PQ2 || FMT == kFmtInt4;  // no residual sites, no WALB2 pair
+  const int r = PLAIN ? 0 : it.r, ks = PLAIN ? 0 : it.k;
   const bool worker = warp < S * P;
   const AreaPlan ap = area_plan(K, S, RB, SIGNED_TABLE, FMT);
   float* partz = reinterpret_cast<float*>(area + ap.partz);
@@ -686,7 +761,7 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
     const TileRec tn = R.sched[j + 1 + tid];
     if (tn.rows) prefetch_l1(R.items + tn.item);
   }
-  build_image<SIGNED_TABLE, PQ2>(xr, K, area, ap);
+  build_image<SIGNED_TABLE, FMT>(xr, K, area, ap);
 
   // the 96 limb words of this lane's group into registers; on lanes with bit
   // 2 set register word w holds group word w ^ 4 (stored so in the image), as
@@ -867,7 +942,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
     }
     if (t.rows == 0 || dead) continue;  // uniform across the CTA
     bool ok;
-    if (FMT == kFmtPq2) ok = do_group<kFmtPq2, false>(t, R, j, st, parity, area, s_z);
+    if (FMT == kFmtPq2 || FMT == kFmtInt4) ok = do_group<FMT, false>(t, R, j, st, parity, area, s_z);
     else ok = t.signed_table ? do_group<FMT, true>(t, R, j, st, parity, area, s_z)
                              : do_group<FMT, false>(t, R, j, st, parity, area, s_z);
     dead = !ok;
@@ -907,6 +982,8 @@ int stream_init() {
       e = cudaFuncSetAttribute(stream_kernel<kFmtPq2>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_max_smem - 1024);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(stream_kernel<kFmtF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_max_smem - 1024);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(stream_kernel<kFmtInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_max_smem - 1024);
     g_err = e;
   });
   if (g_err != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("device initialisation: ") + cudaGetErrorString(g_err));
@@ -977,7 +1054,8 @@ int plan_launch(GroupDesc* groups, int n_groups, bool persistent, int fmt, Strea
     if (!fits) continue;
     for (int j = 0; j < n_groups; ++j) {
       const GroupDesc& g = groups[j];
-      groups[j].signed_table = fmt != kFmtPq2 && off + area_plan(g.K, g.S, g.RB, true, fmt).total <= limit ? 1 : 0;
+      groups[j].signed_table =
+          (fmt == kFmtV1 || fmt == kFmtF32) && off + area_plan(g.K, g.S, g.RB, true, fmt).total <= limit ? 1 : 0;
     }
     L.stages = stages;
     L.rpc = rpc;
@@ -1012,9 +1090,10 @@ static int launch(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream,
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = cooperative ? 1 : 0;
-  const cudaError_t e = prm.fmt == kFmtPq2   ? cudaLaunchKernelEx(&cfg, stream_kernel<kFmtPq2>, prm)
-                        : prm.fmt == kFmtF32 ? cudaLaunchKernelEx(&cfg, stream_kernel<kFmtF32>, prm)
-                                             : cudaLaunchKernelEx(&cfg, stream_kernel<kFmtV1>, prm);
+  const cudaError_t e = prm.fmt == kFmtPq2    ? cudaLaunchKernelEx(&cfg, stream_kernel<kFmtPq2>, prm)
+                        : prm.fmt == kFmtF32  ? cudaLaunchKernelEx(&cfg, stream_kernel<kFmtF32>, prm)
+                        : prm.fmt == kFmtInt4 ? cudaLaunchKernelEx(&cfg, stream_kernel<kFmtInt4>, prm)
+                                              : cudaLaunchKernelEx(&cfg, stream_kernel<kFmtV1>, prm);
   if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("stream_kernel launch: ") + cudaGetErrorString(e));
   return WAL_OK;
 }
@@ -1030,9 +1109,10 @@ int launch_stream(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream)
 int launch_body(StreamParams& prm, const StreamLaunch& L, cudaStream_t stream) {
   if (!prm.t_sched || !prm.t_items || !prm.barrier) return fail(WAL_ERR_ARG, "body launch without tables");
   int per_sm = 0;
-  const void* fn = prm.fmt == kFmtPq2   ? reinterpret_cast<const void*>(stream_kernel<kFmtPq2>)
-                   : prm.fmt == kFmtF32 ? reinterpret_cast<const void*>(stream_kernel<kFmtF32>)
-                                        : reinterpret_cast<const void*>(stream_kernel<kFmtV1>);
+  const void* fn = prm.fmt == kFmtPq2    ? reinterpret_cast<const void*>(stream_kernel<kFmtPq2>)
+                   : prm.fmt == kFmtF32  ? reinterpret_cast<const void*>(stream_kernel<kFmtF32>)
+                   : prm.fmt == kFmtInt4 ? reinterpret_cast<const void*>(stream_kernel<kFmtInt4>)
+                                         : reinterpret_cast<const void*>(stream_kernel<kFmtV1>);
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, L.threads, L.smem);
   if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("occupancy query: ") + cudaGetErrorString(e));
   if (per_sm < 1 || L.grid > per_sm * num_sms())

@@ -15,8 +15,10 @@ constexpr int kMaxItems = 16;
 //          weights); `codes` then points at the block buffer, k = r = 0;
 //  kFmtF32 layout v1 with FP32 scales: {alpha, beta} as two floats per
 //          (row, group) (alpha alone when k = 0) and FP32 per-rank scales (a
-//          prepared RC1 matrix); `scales` and `lr` then point at floats.
-enum : int { kFmtV1 = 0, kFmtPq2 = 1, kFmtF32 = 2 };
+//          prepared RC1 matrix); `scales` and `lr` then point at floats;
+//  kFmtInt4 INT4/g128 (the LM head): `codes` points at the nibble plane
+//          uint8 [N][K/2] (offset 8), `scales` at fp16 d [N][K/128], k = r = 0.
+enum : int { kFmtV1 = 0, kFmtPq2 = 1, kFmtF32 = 2, kFmtInt4 = 3 };
 
 // One product y = W x.
 struct StreamItem {
@@ -67,7 +69,7 @@ struct StreamParams {
   uint32_t area_off;          // shared-memory offset of the per-group area
   unsigned int* barrier;      // grid-barrier counter (zeroed before the launch), body pass only
   int32_t* status;            // workspace status word (may be NULL)
-  int fmt;                    // kFmtV1, kFmtPq2 or kFmtF32
+  int fmt;                    // kFmtV1, kFmtPq2, kFmtF32 or kFmtInt4
 };
 
 struct StreamLaunch {

@@ -137,3 +137,33 @@ def test_base3_sizes():
     assert wal.wal_base3_bytes(1, 128) == 32  # 26 bytes, padded
     assert wal.wal_base3_bytes(2, 5120) == 2048
     assert wal.wal_base3_bytes(1, 100) == 0
+
+
+# ---------------------------------------------------------------------------
+# INT4 LM head and INT3 embedding planes
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K", [(1, 128), (3, 256), (7, 4096), (2, 12288)])
+def test_int4_int3_pack_match_oracle(N, K):
+    from oracle import head_oracle as ho
+    from wal_synth import gen_int3, gen_int4
+    for gen, sizes, pack, ref in ((gen_int4, wal.wal_int4_sizes, wal.wal_int4_pack, ho.int4_pack),
+                                  (gen_int3, wal.wal_int3_sizes, wal.wal_int3_pack, ho.int3_pack)):
+        q, d = gen(N, K, 85, N + K)
+        sc, ss = sizes(N, K)
+        c, s = np.empty(sc, np.uint8), np.empty(ss, np.uint8)
+        pack(q.ctypes.data, d.ctypes.data, N, K, c.ctypes.data, s.ctypes.data)
+        rc, rs = ref(q, d)
+        assert np.array_equal(c, rc) and np.array_equal(s, rs)
+
+
+def test_int_pack_rejects_range():
+    c, s = np.empty(64, np.uint8), np.empty(16, np.uint8)
+    q = np.zeros((1, 128), np.int8)
+    q[0, 9] = 8
+    with pytest.raises(wal.WalError):
+        wal.wal_int4_pack(q.ctypes.data, np.zeros(1, np.uint16).ctypes.data, 1, 128, c.ctypes.data, s.ctypes.data)
+    q[0, 9] = -5
+    c3 = np.empty(48, np.uint8)
+    with pytest.raises(wal.WalError):
+        wal.wal_int3_pack(q.ctypes.data, np.zeros(1, np.uint16).ctypes.data, 1, 128, c3.ctypes.data, s.ctypes.data)
