@@ -288,6 +288,26 @@ def cpu_baseline(specs, n_sample):
 
 
 # ---------------------------------------------------------------------------
+# job timing over replicas
+# ---------------------------------------------------------------------------
+def max_over_ranks(ms, world, device=None):
+    """The largest of the ranks' times (every rank takes part; world 1: itself)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(max_ms, steps, world):
+    """Microseconds per body pass for the whole job: every rank ran `steps`
+    independent passes (replicas), all inside the slowest rank's time."""
+    return max_ms * 1e3 / (steps * world)
+
+
+# ---------------------------------------------------------------------------
 # arms
 # ---------------------------------------------------------------------------
 def run_reference(args):
@@ -356,12 +376,9 @@ def run_wal(args):
     clocks.stop()
     total_ms = t_start.elapsed_time(t_end)
     per_step = np.array([a.elapsed_time(b) for a, b in ev]) * 1e3  # us
-    if world > 1:
-        t = torch.tensor([total_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, device)
     ms_per_step = total_ms / args.steps
-    us_per_pass_job = total_ms * 1e3 / (args.steps * world)
+    us_per_pass_job = job_rate(total_ms, args.steps, world)
     gbs = (wbytes + iobytes) / (ms_per_step * 1e-3) / 1e9
 
     # end to end: pinned host x -> device, body pass, device y -> host, every step
@@ -379,12 +396,8 @@ def run_wal(args):
         w["y_pinned"].copy_(w["y_dev"], non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_us = e2e_ms * 1e3 / (args.steps * world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    e2e_us = job_rate(e2e_ms, args.steps, world)
 
     kernel = time_gate_product(w, device) if rank == 0 else None
     peak, peak_kind = measured_peaks()

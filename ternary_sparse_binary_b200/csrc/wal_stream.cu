@@ -548,7 +548,9 @@ __device__ __forceinline__ bool run_rows(const WarpRing& W, const RingCtx& R, ui
     if (!mbar_wait(R.mbar + st * 8u, parity, R.status)) return false;
     // group index of the chunk's first row (this slice's first group)
     const uint32_t gb0 = (uint32_t)(W.nb + j * C.rpc) * G + 32u * (uint32_t)W.s;
-#pragma unroll
+    // rows one at a time (not unrolled): the loop body stays small enough for
+    // the instruction caches, which measured faster than three unrolled rows
+#pragma unroll 1
     for (int u = 0; u < kMaxRowsPerChunk; ++u) {
       const int i = j * C.rpc + u;
       if (u < C.rpc && i < W.nmine) {  // uniform across the warp
@@ -587,7 +589,7 @@ __device__ __forceinline__ bool run_rows_pq2(const WarpRing& W, const RingCtx& R
   for (int j = 0; j < nc; ++j) {
     const uint32_t sl = R.ring + st * C.bytes;
     if (!mbar_wait(R.mbar + st * 8u, parity, R.status)) return false;
-#pragma unroll
+#pragma unroll 1
     for (int u = 0; u < kMaxRowsPerChunk; ++u) {
       const int i = j * C.rpc + u;
       if (u < C.rpc && i < W.nmine) {  // uniform across the warp
