@@ -119,7 +119,9 @@ int wal_unpack_matrix(const wal_matrix* m, int8_t* T, uint8_t* site_pos, int8_t*
                       uint16_t* alpha, uint16_t* beta, int8_t* U, int8_t* V,
                       wal_stream_t stream);
 
-/* Scratch bytes wal_gemv (M = 1) / wal_gemm_small_m (M <= 16) need. */
+/* Scratch bytes wal_gemv (M = 1) / wal_gemm_small_m (any M) need: the
+ * 256-byte header for M <= 7, the tensor path's X image, WALB2 operand and
+ * split sums from M = 8 on. */
 size_t wal_workspace_bytes(const wal_matrix* m, int M);
 
 /* y[N] = W x for one bf16 activation x[K] (batch 1): the decode-GEMV.
@@ -127,9 +129,10 @@ size_t wal_workspace_bytes(const wal_matrix* m, int M);
 int wal_gemv(const wal_matrix* m, const uint16_t* x, float* y, void* ws, size_t ws_bytes,
              wal_stream_t stream);
 
-/* Y[M][ldy] = X[M][ldx] W^T for 1 <= M.  M <= 16 runs the CUDA-core
- * decode-GEMV family with M accumulators per row; M >= 64 runs the tensor-core
- * path (TMA + tcgen05).  ldx >= K and a multiple of 8; ldy >= N. */
+/* Y[M][ldy] = X[M][ldx] W^T for 1 <= M.  M <= 7 runs the CUDA-core
+ * decode-GEMV, one product per activation row in one launch; M >= 8 runs the
+ * tensor-core path (bulk copies + tcgen05), which decodes each weight once for
+ * up to 256 rows.  ldx >= K and a multiple of 8; ldy >= N. */
 int wal_gemm_small_m(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, int ldy,
                      void* ws, size_t ws_bytes, wal_stream_t stream);
 

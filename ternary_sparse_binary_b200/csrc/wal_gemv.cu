@@ -161,8 +161,14 @@ int launch_rows(const wal_matrix* m, const uint16_t* X, int ldx, float* Y, int l
   return launch_stream(prm, L, stream);
 }
 
+// From 8 activation rows on the tensor-core path is faster: it decodes each
+// weight once for all rows (its time hardly grows with M up to a 256-row
+// tile), while the CUDA-core path streams the weights once per row.  On the
+// 8B gate and down shapes at k = 8, r = 16 the two cross between M = 6 and 8.
+constexpr int kTcMinM = 8;
+
 size_t product_ws_bytes(const wal_matrix* m, int M) {
-  if (M > kMaxItems) return tc_ws_bytes(m, M);
+  if (M >= kTcMinM) return tc_ws_bytes(m, M);
   return ws_layout(0, 0, 0, 0, 0).total;
 }
 
@@ -208,8 +214,8 @@ extern "C" int wal_gemm_small_m(const wal_matrix* m, const uint16_t* X, int M, i
   if (st) return st;
   st = ws_check(ws, ws_bytes, product_ws_bytes(m, M));
   if (st) return st;
-  // more than 16 activation rows: the product is a dense contraction (tensor cores)
-  if (M > kMaxItems) return launch_tc(m, X, M, ldx, Y, ldy, ws_base(ws), (cudaStream_t)stream);
+  // 8 or more activation rows: the product is a dense contraction (tensor cores)
+  if (M >= kTcMinM) return launch_tc(m, X, M, ldx, Y, ldy, ws_base(ws), (cudaStream_t)stream);
   for (int m0 = 0; m0 < M; m0 += kMaxItems) {
     st = launch_rows(m, X, ldx, Y, ldy, m0, std::min(kMaxItems, M - m0), (cudaStream_t)stream,
                      reinterpret_cast<int32_t*>(ws_base(ws)), kFmtV1);

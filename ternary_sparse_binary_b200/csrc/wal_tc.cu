@@ -1,4 +1,4 @@
-// Tensor-core product for batches of more than 16 activation rows
+// Tensor-core product for batches of 8 or more activation rows
 //   Y[M][N] = X[M][K] W^T,   W = alpha*T + beta*R + U diag(s) V^T
 // (WAL-Ternary-8B model card, "Representation").  Only here is the product a
 // dense contraction, so only here do the 5th-generation tensor cores run.

@@ -1,5 +1,5 @@
 """Batch sweep of one product: gate 4096->12288 and down 12288->4096 (k=8,
-r=16), M in {1, 4, 16, 64, 256, 1024}; one JSON line per case.
+r=16), M in {1, 4, 8, 16, 64, 256, 1024}; one JSON line per case.
 
     python -m ternary_sparse_binary_b200.sweep [--reps 20] [--M 64,256]
 
@@ -10,7 +10,7 @@ write) before every call.  Reported per case:
   gbs       algorithmic bytes / time: packed weights + 2 M K (x) + 4 M N (y)
   tflops    algorithmic FLOPs / time: 2 M N K (ternary) + 2 M N G k (sites)
             + 2 M r (N + K) (WALB2)
-  issued_tflops  what the tensor cores execute for M > 16: two K-passes over
+  issued_tflops  what the tensor cores execute for M >= 8: two K-passes over
             the FP16 planes (ternary and residual) + the WALB2 MMA with K = 64
   frac_hbm, frac_tensor  against MEASURED_PEAKS.json (copy GB/s, bf16 burst
             TFLOP/s; FP16 runs at the bf16 rate)
@@ -48,7 +48,7 @@ def peaks():
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--reps", type=int, default=20)
-    ap.add_argument("--M", default="1,4,16,64,256,1024")
+    ap.add_argument("--M", default="1,4,8,16,64,256,1024")
     a = ap.parse_args()
     Ms = [int(v) for v in a.M.split(",")]
     dev = torch.device("cuda", 0)
@@ -84,13 +84,13 @@ def main():
             t = float(np.mean(durs))
             nbytes = payload_bytes(N, K, k, r) + 2 * M * K + 4 * M * N
             flops = 2 * M * N * K + 2 * M * N * G * k + 2 * M * r * (N + K)
-            issued = (2 * (2 if k else 1) * M * N * K + 2 * M * N * 64) if M > 16 else 0
+            issued = (2 * (2 if k else 1) * M * N * K + 2 * M * N * 64) if M >= 8 else 0
             print(json.dumps({
                 "matrix": f"{spec.name} {K}->{N} k={k} r={r}", "M": M, "us": round(t * 1e6, 2),
                 "gbs": round(nbytes / t / 1e9, 1), "frac_hbm": round(nbytes / t / 1e9 / hbm, 4),
                 "tflops": round(flops / t / 1e12, 2), "issued_tflops": round(issued / t / 1e12, 2),
                 "frac_tensor": round(issued / t / 1e12 / tfl, 4) if issued else None,
-                "path": "tcgen05" if M > 16 else "cuda-core", "peaks": kind}), flush=True)
+                "path": "tcgen05" if M >= 8 else "cuda-core", "peaks": kind}), flush=True)
     return 0
 
 

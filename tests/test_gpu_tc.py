@@ -1,4 +1,4 @@
-"""Tensor-core path (more than 16 activation rows) vs the FP64 oracle, through
+"""Tensor-core path (8 or more activation rows) vs the FP64 oracle, through
 the C ABI (needs a B200).
 
 Tolerance as everywhere (oracle.check_tolerance): rel-L2 <= 1e-5 over Y and
@@ -24,6 +24,10 @@ TC_SHAPES = [  # N, K, k, r, M
     (384, 768, 8, 3, 300),     # two activation tiles, the second ragged
     (64, 128, 8, 1, 33),       # a single group, fewer rows than a tile
     (1000, 2176, 8, 8, 64),
+    (1000, 2176, 8, 8, 8),     # the smallest batch on this path
+    (300, 4096, 4, 16, 12),
+    (64, 128, 8, 1, 16),
+    (12288, 4096, 8, 16, 16),  # the gate shape of the batch sweep
 ]
 
 
