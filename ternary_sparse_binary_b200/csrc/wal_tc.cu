@@ -344,20 +344,29 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
     // ---- MMA issuer ----
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(kRows, (uint32_t)p.M_tile);
+      // descriptors of stage 0; a stage step or a 16-column step only moves
+      // the 14-bit start-address field (address / 16), which never carries
+      const uint64_t da0 = sdesc_sw128(a_t(0)), dr0 = sdesc_sw128(a_r(0)), db0 = sdesc_sw128(b_t(0));
+      const uint32_t dstage = stage_bytes >> 4;
       bool ok = true;
+      int s = 0;
+      uint32_t ph = 0u;
       for (int i = 0; i < KBl && ok; ++i) {
-        const int s = i % S;
-        const uint32_t ph = (uint32_t)(i / S) & 1u;
         ok = mbar_wait(b_full(s), ph, p.status) && mbar_wait(a_full(s), ph, p.status);
         if (!ok) break;
         tc_fence_after();
+        const uint64_t so = (uint64_t)((uint32_t)s * dstage);
 #pragma unroll
         for (int kk = 0; kk < kBlockK / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(b_t(s) + 32u * kk);
-          mma_f16(tmem, sdesc_sw128(a_t(s) + 32u * kk), bd, idesc, (i | kk) != 0);
-          if (kHasR) mma_f16(tmem, sdesc_sw128(a_r(s) + 32u * kk), bd, idesc, 1u);
+          const uint64_t bd = db0 + so + 2u * kk;
+          mma_f16(tmem, da0 + so + 2u * kk, bd, idesc, (i | kk) != 0);
+          if (kHasR) mma_f16(tmem, dr0 + so + 2u * kk, bd, idesc, 1u);
         }
         mma_commit(empty(s));
+        if (++s == S) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
       if (ok && has_lr) {
         const int s = KBl % S;
