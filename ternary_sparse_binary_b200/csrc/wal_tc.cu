@@ -43,6 +43,9 @@
 // With few row tiles the K range is split over CTAs (ks splits of whole
 // 128-column groups); each split writes its raw sums and a third launch adds
 // the splits in order and applies 2^-sc_m.  The WALB2 MMA belongs to split 0.
+// Launch 2 is a programmatic dependent launch: it starts while launch 1 runs
+// (the decoders need only the weights), and only its B producer and epilogue
+// wait for launch 1's grid (griddepcontrol.wait).
 // All mbarrier waits are bounded; one that gives up records WAL_ERR_TIMEOUT in
 // the status word and its role stops issuing work.
 #include "wal_internal.h"
@@ -111,6 +114,8 @@ __device__ __forceinline__ int ilog2f_bits(uint32_t b) {
 __global__ void __launch_bounds__(kPrepThreads) tc_prep_kernel(const TcPrepParams p) {
   const int m = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (m == 0 && tid == 0 && p.status) *p.status = 0;
+  // the product launch may start now: its decoders need only the weights
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const bool live = m < p.M;
   const int KB = p.K / kBlockK, n16 = p.K / 16;
   const int mt = m / p.M_tile, row = m % p.M_tile;
@@ -331,6 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
   if (warp == 0) {
     // ---- B producer ----
     if (lane == 0) {
+      // the B tiles are the prep launch's output
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       for (int i = 0; i < n_iter; ++i) {
         const int s = i % S;
         const uint32_t ph = (uint32_t)(i / S) & 1u;
@@ -469,6 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
     }
 
     // ---- epilogue ----
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // the row scales are the prep launch's output
     for (int j = tid - 64; j < p.M_tile; j += 256) {
       const int m = mt * p.M_tile + j;
       const float2 v = m < p.M ? p.scal[m] : make_float2(0.f, 0.f);
@@ -635,14 +643,25 @@ int launch_tc(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, 
   tp.d2_col = m->r > 0 ? P.tmem_cols / 2 : P.tmem_cols;
   tp.tmem_cols = P.tmem_cols;
   tp.status = status;
-  const dim3 grid(P.n_tiles_n * P.ks * P.n_mt);
+  // programmatic dependent launch: the product launch starts while the prep
+  // launch runs; its B producer and epilogue wait for the prep grid
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(P.n_tiles_n * P.ks * P.n_mt);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = P.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   switch (m->k) {
-    case 0: tc_kernel<0><<<grid, kThreads, P.smem, stream>>>(tp); break;
-    case 2: tc_kernel<2><<<grid, kThreads, P.smem, stream>>>(tp); break;
-    case 4: tc_kernel<4><<<grid, kThreads, P.smem, stream>>>(tp); break;
-    default: tc_kernel<8><<<grid, kThreads, P.smem, stream>>>(tp); break;
+    case 0: e = cudaLaunchKernelEx(&cfg, tc_kernel<0>, tp); break;
+    case 2: e = cudaLaunchKernelEx(&cfg, tc_kernel<2>, tp); break;
+    case 4: e = cudaLaunchKernelEx(&cfg, tc_kernel<4>, tp); break;
+    default: e = cudaLaunchKernelEx(&cfg, tc_kernel<8>, tp); break;
   }
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("tc_kernel launch: ") + cudaGetErrorString(e));
   if (P.ks > 1) {
     const size_t total = (size_t)M * m->N;
