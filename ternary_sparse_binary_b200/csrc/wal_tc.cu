@@ -43,9 +43,10 @@
 // With few row tiles the K range is split over CTAs (ks splits of whole
 // 128-column groups); each split writes its raw sums and a third launch adds
 // the splits in order and applies 2^-sc_m.  The WALB2 MMA belongs to split 0.
-// Launch 2 is a programmatic dependent launch: it starts while launch 1 runs
-// (the decoders need only the weights), and only its B producer and epilogue
-// wait for launch 1's grid (griddepcontrol.wait).
+// Launches 2 and 3 are programmatic dependent launches: launch 2 starts while
+// launch 1 runs (the decoders need only the weights), and only its B
+// producer and epilogue wait for launch 1's grid (griddepcontrol.wait);
+// launch 3 is scheduled early and waits for launch 2's whole grid.
 // All mbarrier waits are bounded; one that gives up records WAL_ERR_TIMEOUT in
 // the status word and its role stops issuing work.
 #include "wal_internal.h"
@@ -288,6 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   constexpr bool kHasR = KS > 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the split-sum launch may be scheduled now; it waits for this whole grid
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t b_bytes = (uint32_t)p.M_tile * 128u;
   const uint32_t stage_bytes = kATile * (kHasR ? 2u : 1u) + b_bytes;
@@ -518,6 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
 // Split-K: y[m][n] = 2^-sc_m * sum over splits (in order) of the raw partials.
 __global__ void __launch_bounds__(256) tc_reduce_kernel(const float* __restrict__ part, const float2* __restrict__ scal,
                                                         float* Y, int ldy, int M, int N, int ks) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the partial sums are the product launch's output
   const size_t total = (size_t)M * N;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
     const int m = (int)(i / N), n = (int)(i % N);
@@ -666,8 +670,15 @@ int launch_tc(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, 
   if (P.ks > 1) {
     const size_t total = (size_t)M * m->N;
     const int blocks = (int)std::min<size_t>((total + 255) / 256, 148 * 8);
-    tc_reduce_kernel<<<blocks, 256, 0, stream>>>(tp.part, tp.scal, Y, ldy, M, m->N, P.ks);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t rc = {};
+    rc.gridDim = dim3(blocks);
+    rc.blockDim = dim3(256);
+    rc.stream = stream;
+    rc.attrs = attr;
+    rc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&rc, tc_reduce_kernel, (const float*)tp.part, (const float2*)tp.scal, Y, ldy, M, m->N,
+                           P.ks);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("tc_reduce_kernel launch: ") + cudaGetErrorString(e));
   }
   return WAL_OK;
