@@ -141,6 +141,27 @@ int body_pass_impl(wal_body_plan** plan, int fmt, const wal_matrix* mats, int n_
       // stages renumbered 0, 1, 2, ... (only changes matter to the launch)
       groups[gi].stage = gi == 0 ? 0 : groups[gi - 1].stage + (stage_of[lg.first] != stage_of[lgs[gi - 1].first]);
     }
+    // A group right after a grid barrier may build its x image before the
+    // barrier completes when no product of the stage before writes its x:
+    // no x range of the group meets a y range of that stage.
+    for (size_t gi = 1; gi < groups.size(); ++gi) {
+      groups[gi].xfree = 0;
+      if (groups[gi].stage == groups[gi - 1].stage) continue;
+      bool overlap = false;
+      for (size_t gk = 0; gk < gi && !overlap; ++gk) {
+        if (groups[gk].stage != groups[gi - 1].stage) continue;
+        for (int a = 0; a < groups[gk].n_items && !overlap; ++a) {
+          const StreamItem& w = items[groups[gk].item0 + a];
+          const uintptr_t y0 = (uintptr_t)w.y, y1 = y0 + (uintptr_t)w.N * 4u;
+          for (int b = 0; b < groups[gi].n_items && !overlap; ++b) {
+            const uintptr_t x0 = (uintptr_t)items[groups[gi].item0 + b].x;
+            const uintptr_t x1 = x0 + (uintptr_t)groups[gi].K * 2u;
+            overlap = x0 < y1 && y0 < x1;
+          }
+        }
+      }
+      groups[gi].xfree = overlap ? 0 : 1;
+    }
     StreamLaunch L;
     int st = plan_launch(groups.data(), (int)groups.size(), true, fmt, &L);
     if (st) return st;

@@ -24,9 +24,8 @@
 //    below 2^22 in magnitude (exact when x_j is within 2^-14 of the group
 //    maximum, round-to-nearest-even below that), as three byte limbs per
 //    column, with the group sum of X, the group weight 2^(e_g - 21) and a
-//    table of X (or X then -X) indexed by the residual-site byte, group-major
-//    with an odd stride so the lanes of a warp (one group each) spread over
-//    the banks.  One pass over x and one CTA barrier.
+//    table of X (or X then -X) indexed by the residual-site byte,
+//    group-major.  One pass over x and one CTA barrier.
 //  - Each lane pulls its 96 limb words into registers.  The trit decode
 //    masks each code word once per slot (word & (0x03030303 << 2s) leaves
 //    4^s times the code t + 1 of trit 4b + s in byte b); three dp4a per slot
@@ -202,9 +201,10 @@ __device__ __forceinline__ uint32_t group_dot4(const uint32_t (&wv)[16], const u
 // shared memory: [ring | mbarriers | producer states] then the per-group area
 // ---------------------------------------------------------------------------
 // Site table: per group, the X of its 128 columns (and, in the signed
-// table, their negations after them), group-major with an odd stride so
-// that groups land on different banks.
-__host__ __device__ inline uint32_t table_stride(bool signed_table) { return signed_table ? 257u : 129u; }
+// table, their negations after them), group-major.  The row stride is a
+// multiple of 4 words, so the build writes 16-byte vectors; the site bytes
+// of a warp's lanes are random, so no stride spreads their banks better.
+__host__ __device__ inline uint32_t table_stride(bool signed_table) { return signed_table ? 260u : 132u; }
 
 __host__ __device__ inline uint32_t ring_bytes(int warps, int stages, int rpc, int fmt) {
   return (uint32_t)warps * stages * chunk_geom(rpc, fmt).bytes;
@@ -270,7 +270,7 @@ __device__ __forceinline__ void warp_work(const TileRec& t, const StreamItem* it
 __host__ __device__ inline TileRec tile_record(const GroupDesc& g, const StreamItem* items, int cta) {
   TileRec t = {};
   t.G = (uint8_t)(g.K / kGroup); t.S = (uint8_t)g.S; t.P = (uint8_t)g.P;
-  t.signed_table = (uint8_t)g.signed_table;
+  t.flags = (uint8_t)((g.signed_table ? kTileSigned : 0) | (g.xfree ? kTileXFree : 0));
   t.RB = (uint16_t)g.RB;
   t.stage = (uint16_t)g.stage;
   if (cta >= g.tiles) return t;
@@ -524,6 +524,7 @@ struct RingCtx {
   ChunkGeom C;          // ring chunk geometry
   bool items_global;    // items live in device memory (not kernel parameters)
   int32_t* status;
+  unsigned int* barrier;  // grid-barrier counter (body pass)
 };
 
 // Consume this warp's rows of the current group (ring positions q, q+1, ...);
@@ -657,9 +658,7 @@ __device__ __forceinline__ void build_image(const uint4 (&xr)[kMaxXChunks], int 
     uint32_t m2 = 0u;  // largest |x| bit pattern, two bf16 lanes
 #pragma unroll
     for (int q = 0; q < 4; ++q) m2 = __vmaxu2(m2, pr[q] & 0x7FFF7FFFu);
-    uint32_t mx = max(m2 & 0xFFFFu, m2 >> 16);
-#pragma unroll
-    for (int off = 8; off; off >>= 1) mx = max(mx, __shfl_xor_sync(gmask, mx, off));
+    uint32_t mx = __reduce_max_sync(gmask, max(m2 & 0xFFFFu, m2 >> 16));
     uint32_t emax = mx >> 7;
     emax = emax > 1u ? emax : 1u;  // exponent field of the group maximum (denormals as 1)
     // X = round(x * 2^(127 + kOff - emax)); tiny groups are pre-scaled by 2^64 so the factor stays finite
@@ -673,8 +672,7 @@ __device__ __forceinline__ void build_image(const uint4 (&xr)[kMaxXChunks], int 
       X[q] = (int32_t)(__float_as_uint(fmaf(xv * pre, scl, __uint_as_float(kMagic))) - kMagic);
       sum8 += X[q];
     }
-#pragma unroll
-    for (int off = 8; off; off >>= 1) sum8 += __shfl_xor_sync(gmask, sum8, off);
+    sum8 = __reduce_add_sync(gmask, sum8);
     const int gg = c >> 7, pos = c & 127, h = (c >> 3) & 1;
     // limb image [group][word-in-group][limb][slot] (+4 words of padding per
     // group): byte b of (word wl, limb L, slot q) = limb L of column 16 wl + 4 b + q.
@@ -710,12 +708,13 @@ __device__ __forceinline__ void build_image(const uint4 (&xr)[kMaxXChunks], int 
       gsc_s[gg] = emax > kOff ? __uint_as_float((emax - kOff) << 23) : __uint_as_float(1u << (emax + 22u - kOff));
     }
     // site table: entry e of group gg (e = site byte) at gg * stride + e
-    if (!NO_TABLE) {
-      int32_t* trow = table + (size_t)gg * tstride + pos;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        trow[q] = X[q];
-        if (SIGNED_TABLE) trow[128 + q] = -X[q];
+    if (!NO_TABLE) {  // rows of the table are 16-byte aligned (stride a multiple of 4 words)
+      int4* trow = reinterpret_cast<int4*>(table + (size_t)gg * tstride + pos);
+      trow[0] = make_int4(X[0], X[1], X[2], X[3]);
+      trow[1] = make_int4(X[4], X[5], X[6], X[7]);
+      if (SIGNED_TABLE) {
+        trow[32] = make_int4(-X[0], -X[1], -X[2], -X[3]);
+        trow[33] = make_int4(-X[4], -X[5], -X[6], -X[7]);
       }
     }
   }
@@ -728,9 +727,33 @@ __device__ __forceinline__ void prefetch_l1(const void* p) {
 
 // One group on this CTA (which owns the tile t of it).  Returns false (on
 // every thread) when some wait of the CTA gave up.
+// All CTAs of the launch meet at a grid barrier, in two halves.  Arrive:
+// thread 0 adds one with release semantics (the CTA barrier before it carries
+// the CTA's writes).  Wait: thread 0 polls with acquire loads until `target`
+// = CTAs x barriers so far, and the CTA barrier after it hands the acquired
+// view to every thread.  Between the halves a CTA may do work that reads
+// nothing the other CTAs write before the barrier.  A CTA always waits before
+// it arrives at the next barrier.
+__device__ __forceinline__ void grid_arrive(unsigned int* ctr) {
+  __syncthreads();
+  if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+}
+__device__ __forceinline__ void grid_wait(unsigned int* ctr, unsigned int target, int32_t* status) {
+  if (threadIdx.x == 0)
+    for (uint32_t it = 0; ld_acquire(ctr) < target; ++it)
+      if (it >= kBarrierSpin) {
+        if (status) atomicExch(status, (int32_t)WAL_ERR_TIMEOUT);
+        break;
+      }
+  __syncthreads();
+}
+
+// wait_target != 0: the grid barrier before this group is still open (this
+// CTA has arrived); the x image and the WALB2 phase-1 products are built
+// first, and the barrier is waited for before the rows.
 template <int FMT, bool SIGNED_TABLE>
 __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int j, uint32_t& st, uint32_t& parity,
-                                         unsigned char* area, float* s_z) {
+                                         unsigned char* area, float* s_z, unsigned int wait_target) {
   const int threads = blockDim.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int K = (int)t.G * kGroup, S = t.S, P = t.P, RB = t.RB, rows = t.rows, n0 = t.n0;
   const StreamItem& it = R.items[t.item];
@@ -815,6 +838,7 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
       val = warp_sum(val);
       if (lane == 0) partz[W.s * WAL_MAX_RANK + rho] = val;
     }
+  if (wait_target) grid_wait(R.barrier, wait_target, R.status);
   const uint32_t tab = ptx::smem_u32(area + ap.table) + (uint32_t)g * table_stride(SIGNED_TABLE) * 4u;
   bool ok = true;
   if (PQ2) {
@@ -864,22 +888,6 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
   return all_ok;
 }
 
-// All CTAs of the launch meet here; `target` = CTAs x barriers passed so far.
-// Thread 0 arrives with a release add (the CTA barrier before it carries the
-// CTA's writes) and polls with acquire loads; the CTA barrier after it hands
-// the acquired view to every thread.
-__device__ __forceinline__ void grid_barrier(unsigned int* ctr, unsigned int target, int32_t* status) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
-    for (uint32_t it = 0; ld_acquire(ctr) < target; ++it)
-      if (it >= kBarrierSpin) {
-        if (status) atomicExch(status, (int32_t)WAL_ERR_TIMEOUT);
-        break;
-      }
-  }
-  __syncthreads();
-}
 
 template <int FMT>
 __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_constant__ StreamParams prm) {
@@ -916,6 +924,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
   R.warp = warp;
   R.items_global = table_mode;
   R.status = prm.status;
+  R.barrier = prm.barrier;
   if (lane == 0) {
     for (int st = 0; st < stages; ++st) mbar_init(R.mbar + 8u * st, 1u);
     ptx::mbar_init_fence();
@@ -938,15 +947,23 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
   bool dead = false;
   for (int j = 0; j < n_groups; ++j) {
     const TileRec t = sched[j];
+    unsigned int pending = 0;  // target of a grid barrier this CTA has arrived at but not passed
     if (j > 0 && t.stage != sched[j - 1].stage) {
       ++nbar;
-      grid_barrier(prm.barrier, nbar * gridDim.x, prm.status);
+      grid_arrive(prm.barrier);
+      pending = nbar * gridDim.x;
+      // the x image may be built before the barrier only when the previous
+      // stage does not write this group's x (decided on the host)
+      if (t.rows == 0 || dead || !(t.flags & kTileXFree)) {
+        grid_wait(prm.barrier, pending, prm.status);
+        pending = 0;
+      }
     }
     if (t.rows == 0 || dead) continue;  // uniform across the CTA
     bool ok;
-    if (FMT == kFmtPq2 || FMT == kFmtInt4) ok = do_group<FMT, false>(t, R, j, st, parity, area, s_z);
-    else ok = t.signed_table ? do_group<FMT, true>(t, R, j, st, parity, area, s_z)
-                             : do_group<FMT, false>(t, R, j, st, parity, area, s_z);
+    if (FMT == kFmtPq2 || FMT == kFmtInt4) ok = do_group<FMT, false>(t, R, j, st, parity, area, s_z, pending);
+    else ok = (t.flags & kTileSigned) ? do_group<FMT, true>(t, R, j, st, parity, area, s_z, pending)
+                                      : do_group<FMT, false>(t, R, j, st, parity, area, s_z, pending);
     dead = !ok;
   }
   // never leave with bulk copies in flight: after a wait gave up, wait
@@ -1026,6 +1043,7 @@ int plan_group(StreamItem* items, int n, int K, GroupDesc* out) {
   g.tiles = t;
   g.n_items = n;
   g.signed_table = 1;
+  g.xfree = 0;
   *out = g;
   return WAL_OK;
 }

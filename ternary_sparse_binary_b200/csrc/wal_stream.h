@@ -40,9 +40,13 @@ struct StreamItem {
 struct GroupDesc {
   int K, S, P, RB, rmax, tiles;
   int signed_table;  // +-X table (256 entries) or X table with the sign applied at lookup
+  int xfree;         // the group's x is not written by the previous stage: its x image may be
+                     // built while the grid barrier before it is still open
   int item0, n_items;
   int stage;         // dependency stage (non-decreasing along the group list)
 };
+
+enum : uint8_t { kTileSigned = 1, kTileXFree = 2 };
 
 // What one CTA does in one group (16 bytes; a body pass keeps [CTA][group]
 // of these in device memory and each CTA copies its row into shared memory).
@@ -50,7 +54,7 @@ struct TileRec {
   uint16_t item;   // index into the item table
   uint16_t rows;   // rows of the tile (0: the CTA has no tile in this group)
   int32_t n0;      // first output row of the tile
-  uint8_t G, S, P, signed_table;  // K / 128, slices, phases, table kind
+  uint8_t G, S, P, flags;  // K / 128, slices, phases, kTileSigned | kTileXFree
   uint16_t RB;     // rows per tile of the group
   uint16_t stage;  // dependency stage
 };

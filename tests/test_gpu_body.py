@@ -159,3 +159,37 @@ def test_body27b_full_sampled(body27b, M):
         X, ref = per_m[M]
         assert_parity(y.cpu().numpy().astype(np.float64)[:, rows], ref, X, alpha, f"{s.name} M={M}")
     bp.close()
+
+
+def test_body_dependency_two_stages_back():
+    """Stage 2 reads what stage 0 wrote, across a stage 1 that does not touch
+    it.  The pass builds stage 2's x image while the barrier before it is
+    still open (stage 1 writes no x of stage 2); stage 0's output is complete
+    by then, since every CTA passed the barrier after stage 0.  The buffer
+    starts as NaN, so a read before stage 0's writes shows."""
+    w = wal()
+    NA, KA = 2048, 1024
+    a = gen_components(NA, KA, 0, 0, config_id=61, matrix_index=0)
+    a.T[:] = 0
+    a.T[np.arange(NA), np.arange(NA) % KA] = 1
+    a.alpha[:] = 0x3C00  # fp16 1.0
+    rng = np.random.default_rng(61)
+    xa = bf16_bits_from_f32((rng.uniform(1.0, 2.0, (1, KA)) * rng.choice([-1.0, 1.0], (1, KA))).astype(np.float32))
+    mid = gen_components(3000, 4096, 8, 8, config_id=61, matrix_index=1)   # stage 1, its own x
+    xm = gen_x(4096, 1, 61, 1)
+    b = gen_components(4096, 2 * NA, 8, 8, config_id=61, matrix_index=2)  # stage 2 reads y_A
+    ya = torch.full((NA,), float("nan"), dtype=torch.float32, device="cuda")
+    ym = torch.empty(3000, dtype=torch.float32, device="cuda")
+    yb = torch.empty(4096, dtype=torch.float32, device="cuda")
+    mats = [device_matrix(a), device_matrix(mid), device_matrix(b)]
+    bp = w.BodyPass(mats, [0, 1, 2], [device_bf16(xa), device_bf16(xm), ya.view(torch.int16)], [ya, ym, yb], M=1)
+    for _ in range(3):
+        ya.fill_(float("nan"))
+        bp.run()
+        torch.cuda.synchronize()
+        _status(bp)
+        assert np.array_equal(ya.cpu().numpy().astype(np.float64), oracle.matvec(a, xa[0]))
+        assert_parity(ym.cpu().numpy().astype(np.float64), oracle.matvec(mid, xm[0]), xm[0], mid.alpha, "stage 1")
+        xb_bits = ya.cpu().numpy().view(np.uint16)
+        assert_parity(yb.cpu().numpy().astype(np.float64), oracle.matvec(b, xb_bits), xb_bits, b.alpha, "stage 2")
+    bp.close()
