@@ -296,8 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
   const uint32_t stage_bytes = kATile * (kHasR ? 2u : 1u) + b_bytes;
   const int S = p.stages;
   const uint32_t bars = base + (uint32_t)S * stage_bytes;
-  // barriers: b_full[S], a_full[S], empty[S], acc_full
-  auto b_full = [&](int s) { return bars + 8u * s; };
+  // barriers: [S] (unused), a_full[S], empty[S], acc_full.  a_full(s) completes
+  // when the 128 decoders of the stage's team have arrived and the B tile's
+  // bulk copy (one more arrival, with its bytes) has landed.
   auto a_full = [&](int s) { return bars + 8u * (S + s); };
   auto empty = [&](int s) { return bars + 8u * (2 * S + s); };
   const uint32_t acc_full = bars + 8u * (3 * S);
@@ -320,8 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(b_full(s), 1);
-      mbar_init(a_full(s), 128);
+      mbar_init(a_full(s), 129);  // 128 decoder arrivals + the B tile's arrival with its bytes
       mbar_init(empty(s), 1);
     }
     mbar_init(acc_full, 1);
@@ -346,8 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
         const uint32_t ph = (uint32_t)(i / S) & 1u;
         if (!mbar_wait(empty(s), ph ^ 1u, p.status)) break;
         const char* src = i < KBl ? p.xt + ((size_t)mt * KB + kb0 + i) * b_bytes : p.zt + (size_t)mt * b_bytes;
-        mbar_arrive_expect_tx(b_full(s), b_bytes);
-        bulk_g2s(b_t(s), src, b_bytes, b_full(s));
+        mbar_arrive_expect_tx(a_full(s), b_bytes);
+        bulk_g2s(b_t(s), src, b_bytes, a_full(s));
       }
     }
   } else if (warp == 1) {
@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
       int s = 0;
       uint32_t ph = 0u;
       for (int i = 0; i < KBl && ok; ++i) {
-        ok = mbar_wait(b_full(s), ph, p.status) && mbar_wait(a_full(s), ph, p.status);
+        ok = mbar_wait(a_full(s), ph, p.status);
         if (!ok) break;
         tc_fence_after();
         const uint64_t so = (uint64_t)((uint32_t)s * dstage);
@@ -381,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
       if (ok && has_lr) {
         const int s = KBl % S;
         const uint32_t ph = (uint32_t)(KBl / S) & 1u;
-        ok = mbar_wait(b_full(s), ph, p.status) && mbar_wait(a_full(s), ph, p.status);
+        ok = mbar_wait(a_full(s), ph, p.status);
         if (ok) {
           tc_fence_after();
           for (int kk = 0; kk < (2 * p.r + 15) / 16; ++kk)
