@@ -249,7 +249,7 @@ struct WarpRing {
 };
 
 // What warp `warp` does for tile record t of product `it` (nmine = 0: nothing).
-// `it` is read only when the record has rows.  The P warps of a slice take
+// `it` is read only when this warp has rows.  The P warps of a slice take
 // contiguous blocks of ceil(rows / P) rows.
 __device__ __forceinline__ void warp_work(const TileRec& t, const StreamItem* it, int warp, WarpRing& W) {
   W.codes = nullptr; W.sites = nullptr; W.scales = nullptr;
@@ -258,12 +258,15 @@ __device__ __forceinline__ void warp_work(const TileRec& t, const StreamItem* it
   W.nb = t.n0;
   W.G = t.G; W.K = (int)t.G * kGroup; W.k = 0;
   if (t.rows == 0 || warp >= (int)t.S * t.P) return;
-  W.codes = it->codes; W.sites = it->sites; W.scales = it->scales; W.k = it->k;
   W.s = warp % t.S;
   const int p = warp / t.S, m = ((int)t.rows + t.P - 1) / t.P;
   W.r0 = p * m;
   W.nb = t.n0 + W.r0;
   W.nmine = max(0, min(m, (int)t.rows - W.r0));
+  // the producer skips the groups where this warp has no rows without a
+  // round trip to memory
+  if (W.nmine == 0) return;
+  W.codes = it->codes; W.sites = it->sites; W.scales = it->scales; W.k = it->k;
 }
 
 // Host and device: the tile record of CTA `cta` in group g.
