@@ -34,13 +34,16 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 200 body passes on the GPU, 20 oracle samples on the CPU)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["wal", "reference"], default="wal")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-matrices", type=int, default=4)
     ap.add_argument("--workload", choices=["body8b", "pq2_body8b"], default="body8b")
     a = ap.parse_args()
+    if a.steps is None:
+        a.steps = 20 if a.impl == "reference" else 200
     global WORKLOAD
     WORKLOAD = a.workload
     return a
@@ -85,34 +88,84 @@ def measured_peaks():
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock and clock-event reasons sampled every few milliseconds in a
+    thread through NVML (read-only queries; the library nvidia-smi reads),
+    each sample stamped with time.monotonic(), so that the summary keeps only
+    the samples taken inside the timed window.  Falls back to an
+    `nvidia-smi -lms` child when the NVML binding is missing."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.rows = []
+    def __init__(self, device_index, period_s=0.002):
+        self.dev = device_index
+        self.period = period_s
+        self.rows = []  # (t, sm_mhz, sm_max_mhz, [reason names])
         self.proc = None
         self.thread = None
+        self.halt = threading.Event()
+        self.source = "none"
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        uuid = getattr(torch.cuda.get_device_properties(self.dev), "uuid", None)
+        if uuid is not None:
+            try:
+                return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(uuid))
+            except Exception:
+                pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.dev)
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+            nv, h = self._nvml_handle()
+        except Exception:
+            return self._start_smi()
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        self.source = "nvml"
+
+        def loop():
+            while not self.halt.is_set():
+                t = time.monotonic()
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    mask = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except Exception:
+                    break
+                self.rows.append((t, float(sm), float(smax), [n for n, b in bits.items() if mask & b]))
+                time.sleep(self.period)
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
+
+    def _start_smi(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.source = "nvidia-smi"
+
+        def read():
+            for line in self.proc.stdout:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    self.rows.append((time.monotonic(), float(parts[1]), float(parts[2]) if parts[2].replace(
+                        ".", "").isdigit() else float("nan"),
+                        [n for n, v in zip(self.NAMES, parts[5:9]) if v.lower() == "active"]))
+        self.thread = threading.Thread(target=read, daemon=True)
         self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                self.rows.append(parts)
-
     def stop(self):
+        self.halt.set()
         if self.proc:
             self.proc.terminate()
             try:
@@ -122,15 +175,18 @@ class ClockSampler:
         if self.thread:
             self.thread.join(timeout=2)
 
-    def summary(self):
-        if not self.rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in self.rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
-        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(self.rows)}
+    def summary(self, t0=None, t1=None):
+        """Samples with t0 <= t <= t1 (all of them without a window)."""
+        rows = [r for r in self.rows if (t0 is None or r[0] >= t0) and (t1 is None or r[0] <= t1)]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0,
+                    "source": self.source}
+        sm = [r[1] for r in rows]
+        smax = [r[2] for r in rows if r[2] == r[2]]
+        return {"sm_mhz": float(np.median(sm)), "sm_min_mhz": float(min(sm)),
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted({n for r in rows for n in r[3]}), "samples": len(rows), "source": self.source,
+                "window_ms": round(1e3 * (rows[-1][0] - rows[0][0]), 1)}
 
 
 # ---------------------------------------------------------------------------
@@ -357,13 +413,14 @@ def run_wal(args):
 
     clocks = ClockSampler(local_rank)
     clocks.start()
-    time.sleep(0.3)
+    time.sleep(0.05)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    h_start = time.monotonic()
     t_start.record(stream)
     for i in range(args.steps):
         ev[i][0].record(stream)
@@ -371,6 +428,7 @@ def run_wal(args):
         ev[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
+    h_end = time.monotonic()
     if world > 1:
         dist.barrier()
     clocks.stop()
@@ -430,7 +488,7 @@ def run_wal(args):
                               "scope": "whole body pass (graph): packed weights + x + y per pass / ms per pass"},
             "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks.summary(),
+            "clocks": clocks.summary(h_start, h_end),
         }
         if cb:
             line["cpu_baseline"] = cb
