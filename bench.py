@@ -29,6 +29,7 @@ METRIC = "µs per 8B body pass (batch 1) + weight GB/s as % of B200 HBM roofline
 UNIT = "us/pass"
 WORKLOAD = "body8b"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, DGX figure
 
 
 def parse():
@@ -485,6 +486,7 @@ def run_wal(args):
                          "bytes_per_launch": kernel["bytes_per_launch"], "us_per_launch": kernel["us_per_launch"],
                          "timing": "CUDA events around each launch on its stream, L2 flushed between launches"},
             "pass_roofline": {"achieved": gbs, "unit": "GB/s", "frac": gbs / peak,
+                              "frac_of_nominal_8tbs": gbs / NOMINAL_HBM_GBS,
                               "scope": "whole body pass (graph): packed weights + x + y per pass / ms per pass"},
             "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
