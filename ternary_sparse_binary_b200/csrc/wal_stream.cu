@@ -49,6 +49,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <vector>
 
 namespace wal {
 
@@ -215,9 +216,15 @@ __host__ __device__ inline uint32_t area_offset(int warps, int stages, int rpc, 
 struct AreaPlan {
   uint32_t table, limbs, part, xgsum, gsc, partz, ubuf, vstage, total;
 };
+// Row pitch of the lane partials: RB rounded up to odd, so that the 32 lanes'
+// stores of one row (stride pitch words) fall in 32 different banks.
+// Partials of a tile: [slice][lane][pitch] with lane partials (a row's 32
+// lanes are summed in the combine), else [slice][RB] (summed by a warp
+// butterfly in the row loop).
+__host__ __device__ inline uint32_t part_pitch(int RB) { return (uint32_t)RB | 1u; }
 // Carve-up of the per-group area (offsets relative to the area base).  A
 // PQ2_0 group has no site table and no WALB2 pair.
-__host__ __device__ inline AreaPlan area_plan(int K, int S, int RB, bool signed_table, int fmt) {
+__host__ __device__ inline AreaPlan area_plan(int K, int S, int RB, bool signed_table, int fmt, bool lanes) {
   AreaPlan p;
   uint32_t off = 0;
   auto take = [&](uint32_t bytes) { uint32_t o = off; off = (off + bytes + 15u) & ~15u; return o; };
@@ -225,7 +232,7 @@ __host__ __device__ inline AreaPlan area_plan(int K, int S, int RB, bool signed_
   const bool v1 = fmt == kFmtV1 || fmt == kFmtF32;
   p.table = take(v1 ? G * table_stride(signed_table) * 4u : 0u);
   p.limbs = take(G * kLimbStride * 4u);
-  p.part = take((uint32_t)S * RB * 4u);  // one partial per (slice, row)
+  p.part = take((uint32_t)S * (lanes ? 32u * part_pitch(RB) : (uint32_t)RB) * 4u);
   p.xgsum = take(G * 4u);
   p.gsc = take(G * 4u);
   p.partz = take(v1 ? (uint32_t)S * WAL_MAX_RANK * 4u : 0u);
@@ -273,7 +280,8 @@ __device__ __forceinline__ void warp_work(const TileRec& t, const StreamItem* it
 __host__ __device__ inline TileRec tile_record(const GroupDesc& g, const StreamItem* items, int cta) {
   TileRec t = {};
   t.G = (uint8_t)(g.K / kGroup); t.S = (uint8_t)g.S; t.P = (uint8_t)g.P;
-  t.flags = (uint8_t)((g.signed_table ? kTileSigned : 0) | (g.xfree ? kTileXFree : 0));
+  t.flags = (uint8_t)((g.signed_table ? kTileSigned : 0) | (g.xfree ? kTileXFree : 0) |
+                      (g.lane_parts ? kTileLaneParts : 0));
   t.RB = (uint16_t)g.RB;
   t.stage = (uint16_t)g.stage;
   if (cta >= g.tiles) return t;
@@ -533,13 +541,26 @@ struct RingCtx {
 // Consume this warp's rows of the current group (ring positions q, q+1, ...);
 // after each chunk lane 0 refills the slot with the producer's next chunk.
 // False when a wait gave up.
+// A row's value leaves the row loop as this lane's partial (summed in the
+// combine, no dependent chain in the loop) or, where the lane buffer does not
+// fit, as the warp's butterfly sum stored by lane 0.  Both give the same bits.
+__device__ __forceinline__ void store_row(float* dst, float v, bool lanes, int lane) {
+  if (lanes) {
+    *dst = v;
+  } else {
+    v = warp_sum(v);
+    if (lane == 0) *dst = v;
+  }
+}
+
 template <int KS, bool SIGNED_TABLE, int FMT>
 __device__ __forceinline__ bool run_rows(const WarpRing& W, const RingCtx& R, uint32_t& st, uint32_t& parity, int RB,
                                          int lane, bool active, uint32_t hsw, const uint32_t (&lb)[8][kLimbWords],
-                                         int32_t xs, float gsc, uint32_t tab, float* part) {
+                                         int32_t xs, float gsc, uint32_t tab, float* part, bool lanes) {
   const ChunkGeom& C = R.C;
   const int nc = (W.nmine + C.rpc - 1) / C.rpc;
-  float* mine = part + W.s * RB + W.r0;  // this warp's row i at mine[i]
+  // row i of this warp: lane partials at mine[i], or the warp's sum at mine[i] (lane 0)
+  float* mine = lanes ? part + (uint32_t)(W.s * 32 + lane) * part_pitch(RB) + W.r0 : part + W.s * RB + W.r0;
   const uint32_t kb = site_bytes(KS), sb = scale_bytes<FMT>(KS);
   const bool one = W.one_slice();
   const uint32_t G = (uint32_t)W.G;
@@ -563,8 +584,7 @@ __device__ __forceinline__ bool run_rows(const WarpRing& W, const RingCtx& R, ui
         const uint32_t arow = sl + C.scales + (uint32_t)u * ap + ((gb * sb) & 15u);
         const float v =
             row_value<KS, SIGNED_TABLE, FMT>(sl + (uint32_t)u * cp, srow, arow, lane, hsw, lb, xs, gsc, tab);
-        const float tot = warp_sum(active ? v : 0.f);  // fixed butterfly order: reproducible
-        if (lane == 0) mine[i] = tot;
+        store_row(mine + i, active ? v : 0.f, lanes, lane);
       }
     }
     __syncwarp();  // every lane has consumed the slot before it is refilled
@@ -583,10 +603,10 @@ __device__ __forceinline__ bool run_rows(const WarpRing& W, const RingCtx& R, ui
 // run_rows for PQ2_0 rows: lane l takes block l of the warp's K-slice.
 __device__ __forceinline__ bool run_rows_pq2(const WarpRing& W, const RingCtx& R, uint32_t& st, uint32_t& parity,
                                              int RB, int lane, bool active, const uint32_t (&lb)[8][kLimbWords],
-                                             int32_t xs, float gsc, float* part) {
+                                             int32_t xs, float gsc, float* part, bool lanes) {
   const ChunkGeom& C = R.C;
   const int nc = (W.nmine + C.rpc - 1) / C.rpc;
-  float* mine = part + W.s * RB + W.r0;
+  float* mine = lanes ? part + (uint32_t)(W.s * 32 + lane) * part_pitch(RB) + W.r0 : part + W.s * RB + W.r0;
   const bool one = W.one_slice();
   const uint32_t G = (uint32_t)W.G, rowb = G * kPq2Block;
 #pragma unroll 1
@@ -602,8 +622,7 @@ __device__ __forceinline__ bool run_rows_pq2(const WarpRing& W, const RingCtx& R
                                  : sl + (uint32_t)u * kPq2Pitch +
                                        ((((uint32_t)(W.nb + i) * G + 32u * (uint32_t)W.s) * kPq2Block) & 15u);
         const float v = pq2_row_value(row + kPq2Block * (uint32_t)lane, lb, xs, gsc);
-        const float tot = warp_sum(active ? v : 0.f);
-        if (lane == 0) mine[i] = tot;
+        store_row(mine + i, active ? v : 0.f, lanes, lane);
       }
     }
     __syncwarp();
@@ -724,6 +743,20 @@ __device__ __forceinline__ void build_image(const uint4 (&xr)[kMaxXChunks], int 
   __syncthreads();
 }
 
+// Sum of the 32 lane partials of one row (lane l at p[l * pitch]) as the
+// pairwise tree of a xor-16, 8, 4, 2, 1 butterfly, so that a row's value is
+// the same as a warp butterfly would give lane 0.
+__device__ __forceinline__ float lane_sum(const float* p, uint32_t pitch) {
+  float v[32];
+#pragma unroll
+  for (int l = 0; l < 32; ++l) v[l] = p[(uint32_t)l * pitch];
+#pragma unroll
+  for (int w = 16; w; w >>= 1)
+#pragma unroll
+    for (int l = 0; l < w; ++l) v[l] += v[l + w];
+  return v[0];
+}
+
 __device__ __forceinline__ void prefetch_l1(const void* p) {
   asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
@@ -766,7 +799,8 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
   constexpr bool PLAIN = PQ2 || FMT == kFmtInt4;  // no residual sites, no WALB2 pair
   const int r = PLAIN ? 0 : it.r, ks = PLAIN ? 0 : it.k;
   const bool worker = warp < S * P;
-  const AreaPlan ap = area_plan(K, S, RB, SIGNED_TABLE, FMT);
+  const bool lanes = (t.flags & kTileLaneParts) != 0;
+  const AreaPlan ap = area_plan(K, S, RB, SIGNED_TABLE, FMT, lanes);
   float* partz = reinterpret_cast<float*>(area + ap.partz);
   float* part = reinterpret_cast<float*>(area + ap.part);
   uint32_t* ubuf = reinterpret_cast<uint32_t*>(area + ap.ubuf);
@@ -845,13 +879,13 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
   const uint32_t tab = ptx::smem_u32(area + ap.table) + (uint32_t)g * table_stride(SIGNED_TABLE) * 4u;
   bool ok = true;
   if (PQ2) {
-    if (worker) ok = run_rows_pq2(W, R, st, parity, RB, lane, active, lb, xs, gsc, part);
+    if (worker) ok = run_rows_pq2(W, R, st, parity, RB, lane, active, lb, xs, gsc, part, lanes);
   } else if (worker) {
     switch (ks) {
-      case 8: ok = run_rows<8, SIGNED_TABLE, FMT>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
-      case 4: ok = run_rows<4, SIGNED_TABLE, FMT>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
-      case 2: ok = run_rows<2, SIGNED_TABLE, FMT>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
-      default: ok = run_rows<0, SIGNED_TABLE, FMT>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part); break;
+      case 8: ok = run_rows<8, SIGNED_TABLE, FMT>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part, lanes); break;
+      case 4: ok = run_rows<4, SIGNED_TABLE, FMT>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part, lanes); break;
+      case 2: ok = run_rows<2, SIGNED_TABLE, FMT>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part, lanes); break;
+      default: ok = run_rows<0, SIGNED_TABLE, FMT>(W, R, st, parity, RB, lane, active, hsw, lb, xs, gsc, tab, part, lanes); break;
     }
   }
 
@@ -876,9 +910,10 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
     s_z[tid] = s * a;
   }
   __syncthreads();
+  const uint32_t pp = part_pitch(RB);
   for (int rl = tid; rl < rows; rl += threads) {
     float acc = 0.f;
-    for (int s2 = 0; s2 < S; ++s2) acc += part[s2 * RB + rl];
+    for (int s2 = 0; s2 < S; ++s2) acc += lanes ? lane_sum(part + (uint32_t)s2 * 32u * pp + rl, pp) : part[s2 * RB + rl];
     if (r > 0) {
       const uint32_t uw = ubuf[rl];
       float lr = 0.f;
@@ -1047,6 +1082,7 @@ int plan_group(StreamItem* items, int n, int K, GroupDesc* out) {
   g.n_items = n;
   g.signed_table = 1;
   g.xfree = 0;
+  g.lane_parts = 1;
   *out = g;
   return WAL_OK;
 }
@@ -1067,18 +1103,29 @@ int plan_launch(GroupDesc* groups, int n_groups, bool persistent, int fmt, Strea
     const uint32_t off = soff + sched_bytes;
     uint32_t need = off;
     bool fits = true;
+    // per group, the first area that fits: lane partials before the signed
+    // table (the lane partials take the dependent reduction out of every row)
+    std::vector<int> pick((size_t)n_groups, 0);
     for (int j = 0; j < n_groups && fits; ++j) {
       const GroupDesc& g = groups[j];
-      const uint32_t as = area_plan(g.K, g.S, g.RB, true, fmt).total, au = area_plan(g.K, g.S, g.RB, false, fmt).total;
-      if (off + as <= limit) need = std::max(need, off + as);
-      else if (off + au <= limit) need = std::max(need, off + au);
-      else fits = false;
+      const bool v1 = fmt == kFmtV1 || fmt == kFmtF32;
+      int chosen = -1;
+      for (int c = 0; c < 4 && chosen < 0; ++c) {  // c: bit 1 = warp sums, bit 0 = unsigned table
+        if (v1 || !(c & 1)) {
+          const uint32_t a = area_plan(g.K, g.S, g.RB, v1 && !(c & 1), fmt, !(c & 2)).total;
+          if (off + a <= limit) {
+            chosen = c;
+            need = std::max(need, off + a);
+          }
+        }
+      }
+      if (chosen < 0) fits = false;
+      else pick[j] = chosen;
     }
     if (!fits) continue;
     for (int j = 0; j < n_groups; ++j) {
-      const GroupDesc& g = groups[j];
-      groups[j].signed_table =
-          (fmt == kFmtV1 || fmt == kFmtF32) && off + area_plan(g.K, g.S, g.RB, true, fmt).total <= limit ? 1 : 0;
+      groups[j].signed_table = (fmt == kFmtV1 || fmt == kFmtF32) && !(pick[j] & 1) ? 1 : 0;
+      groups[j].lane_parts = !(pick[j] & 2);
     }
     L.stages = stages;
     L.rpc = rpc;

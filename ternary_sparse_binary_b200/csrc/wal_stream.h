@@ -42,11 +42,13 @@ struct GroupDesc {
   int signed_table;  // +-X table (256 entries) or X table with the sign applied at lookup
   int xfree;         // the group's x is not written by the previous stage: its x image may be
                      // built while the grid barrier before it is still open
+  int lane_parts;    // rows leave one partial per lane (summed in the combine) rather than a
+                     // warp-reduced one; set where the 32x larger buffer fits shared memory
   int item0, n_items;
   int stage;         // dependency stage (non-decreasing along the group list)
 };
 
-enum : uint8_t { kTileSigned = 1, kTileXFree = 2 };
+enum : uint8_t { kTileSigned = 1, kTileXFree = 2, kTileLaneParts = 4 };
 
 // What one CTA does in one group (16 bytes; a body pass keeps [CTA][group]
 // of these in device memory and each CTA copies its row into shared memory).
@@ -54,7 +56,7 @@ struct TileRec {
   uint16_t item;   // index into the item table
   uint16_t rows;   // rows of the tile (0: the CTA has no tile in this group)
   int32_t n0;      // first output row of the tile
-  uint8_t G, S, P, flags;  // K / 128, slices, phases, kTileSigned | kTileXFree
+  uint8_t G, S, P, flags;  // K / 128, slices, phases, kTileSigned | kTileXFree | kTileLaneParts
   uint16_t RB;     // rows per tile of the group
   uint16_t stage;  // dependency stage
 };

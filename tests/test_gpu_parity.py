@@ -90,6 +90,23 @@ def test_deterministic_reruns():
     assert np.array_equal(run_gemv(pm, xd), run_gemv(pm, xd))
 
 
+def test_tall_matrix_both_row_reductions():
+    """162800 x 128: a row block of 1100 rows, whose per-lane partials do not
+    fit in shared memory beside the weight ring, so each row is reduced by a
+    warp butterfly in the row loop.  Its first 1000 rows as a matrix of their
+    own keep per-lane partials, summed in the combine by the same tree: the
+    two must agree bit for bit, and the tall product must meet the oracle."""
+    N, K, n = 148 * 1100, 128, 1000
+    c = gen_components(N, K, 8, 4, config_id=97, matrix_index=1)
+    x = gen_x(K, 1, 97, 1)[0]
+    xd = device_bf16(x)
+    y = run_gemv(device_matrix(c), xd)
+    assert_parity(y, oracle.matvec(c, x), x, c.alpha, f"{N}x{K}")
+    head = Components(n, K, 8, 4, c.T[:n], c.site_pos[:n], c.site_sign[:n], c.alpha[:n], c.beta[:n], c.U[:n],
+                      c.V, c.lr_scale)
+    assert np.array_equal(run_gemv(device_matrix(head), xd), y[:n])
+
+
 def test_wide_dynamic_range_x():
     """x spanning 2^-40 .. 2^20 inside one group: small entries are rounded in
     the fixed-point image, which the tolerance absorbs."""
