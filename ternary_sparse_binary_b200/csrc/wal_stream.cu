@@ -14,7 +14,7 @@
 // columns; a group uses S slices x P phases warps.
 //  - Weights stream through a per-warp TMA ring that runs ahead across group
 //    and stage boundaries (the weights do not depend on x): lane 0 of each
-//    warp keeps `stages` chunks of two rows in flight, one bulk copy each for
+//    warp keeps `stages` chunks of 2-3 rows in flight, one bulk copy each for
 //    a row's code bytes (32 lanes x 32 B), residual-site bytes and
 //    {alpha, beta} words, completing on an mbarrier per ring slot.  While a
 //    CTA waits at the grid barrier its ring already fills with the next
@@ -35,10 +35,12 @@
 //    (exact).  alpha and beta are applied in FP32 and the group weight once.
 //    The WALB2 phase-1 products V_r^T x go through the same path: a row of
 //    V is a ternary row without zeros, its bits spread into 2-bit codes.
-//  - Each row's lane partials are summed across the warp by a fixed
-//    butterfly; after the rows one thread per output row adds the slices in
-//    order, and the WALB2 phase-2 term sum_r U[n, r] z_r joins in the single
-//    store.
+//  - Each lane stores its row partial to shared memory; after the rows one
+//    thread per output row sums the row's 32 lane partials (the pairwise tree
+//    of a xor-16 .. 1 butterfly) and the slices in order, and the WALB2
+//    phase-2 term sum_r U[n, r] z_r joins in the single store.  Where the
+//    lane buffer does not fit (very large row blocks), the row loop sums the
+//    lanes with that butterfly itself; the bits are the same.
 // Results are bitwise reproducible: no atomics in the arithmetic, fixed
 // reduction orders.  Every wait (mbarrier, grid barrier) is bounded; one that
 // gives up records WAL_ERR_TIMEOUT in the status word and the waiter moves on.
