@@ -216,7 +216,7 @@ struct ProdState;  // defined below
 __host__ __device__ inline uint32_t area_offset(int warps, int stages, int rpc, int fmt);
 
 struct AreaPlan {
-  uint32_t table, limbs, part, xgsum, gsc, partz, ubuf, vstage, total;
+  uint32_t table, limbs, part, xgsum, gsc, partz, ubuf, vstage, lrs, total;
 };
 // Row pitch of the lane partials: RB rounded up to odd, so that the 32 lanes'
 // stores of one row (stride pitch words) fall in 32 different banks.
@@ -241,6 +241,7 @@ __host__ __device__ inline AreaPlan area_plan(int K, int S, int RB, bool signed_
   p.ubuf = take(v1 ? (uint32_t)RB * 4u : 0u);
   // V bit planes of the first P ranks (each of the P phases of a slice takes one): P * K / 8 bytes
   p.vstage = take(v1 ? (uint32_t)(kMaxWarps / S) * (uint32_t)K / 8u : 0u);
+  p.lrs = take(v1 ? WAL_MAX_RANK * 4u : 0u);  // the per-rank scales (FP16 or FP32)
   p.total = off;
   return p;
 }
@@ -817,6 +818,9 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
       cp_async4_zfill(ptx::smem_u32(ubuf + rl), it.ubits + (size_t)(n0 + rl) * ((r + 31) / 32), 4u);
     for (int i = tid; i < rv * (K / 128); i += threads)
       cp_async16(reinterpret_cast<void*>(area + ap.vstage + 16u * i), it.vbits + 4 * i);
+    // per-rank scales for the combine (the buffer is padded to 16 bytes)
+    if (tid < (r * (FMT == kFmtF32 ? 4 : 2) + 15) / 16)
+      cp_async16(reinterpret_cast<void*>(area + ap.lrs + 16u * tid), reinterpret_cast<const char*>(it.lr) + 16 * tid);
   }
   cp_async_commit();
 
@@ -908,7 +912,8 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
   if (tid < r) {
     float a = 0.f;
     for (int s2 = 0; s2 < S; ++s2) a += partz[s2 * WAL_MAX_RANK + tid];
-    const float s = FMT == kFmtF32 ? reinterpret_cast<const float*>(it.lr)[tid] : fp16_bits_to_float(it.lr[tid]);
+    const float s = FMT == kFmtF32 ? reinterpret_cast<const float*>(area + ap.lrs)[tid]
+                                   : fp16_bits_to_float(reinterpret_cast<const uint16_t*>(area + ap.lrs)[tid]);
     s_z[tid] = s * a;
   }
   __syncthreads();
