@@ -28,6 +28,9 @@
  *   u_bits   uint32[N][ceil(r/32)]  bit (rho % 32) of word rho/32 set <=> U[n][rho] = -1
  *   v_bits   uint32[r][K/32]   bit (j % 32) of word j/32 set <=> V[j][rho] = -1
  *   lr_scale uint16[r]         fp16 bits of s_rho
+ * Each buffer spans the size wal_packed_sizes returns (its payload rounded
+ * up to a multiple of 16 bytes) and its padding bytes are zero: the kernels
+ * read whole aligned 16-byte words of every buffer.
  * Activations are bf16 bit patterns, row-major X[M][ldx]; outputs are fp32,
  * row-major Y[M][ldy], overwritten (never accumulated into).
  *
