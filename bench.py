@@ -175,6 +175,12 @@ class ClockSampler:
                 self.proc.kill()
         if self.thread:
             self.thread.join(timeout=2)
+        if self.source == "nvml" and not (self.thread and self.thread.is_alive()):
+            try:
+                import pynvml
+                pynvml.nvmlShutdown()
+            except Exception:
+                pass
 
     def summary(self, t0=None, t1=None):
         """Samples with t0 <= t <= t1 (all of them without a window)."""
