@@ -167,3 +167,36 @@ def test_int_pack_rejects_range():
     c3 = np.empty(48, np.uint8)
     with pytest.raises(wal.WalError):
         wal.wal_int3_pack(q.ctypes.data, np.zeros(1, np.uint16).ctypes.data, 1, 128, c3.ctypes.data, s.ctypes.data)
+
+
+@pytest.mark.parametrize("N,K,k,r1,r2", [(512, 1024, 8, 4, 4), (37, 384, 0, 1, 0), (9, 17408, 2, 16, 16),
+                                         (64, 128, 4, 0, 3)])
+def test_rc1_sizes_match_oracle_planes(N, K, k, r1, r2):
+    """The library's RC1 plane sizes equal the byte counts of the oracle's own
+    canonical and prepared planes (each zero-padded to 16 bytes)."""
+    from oracle import rc1_oracle as rc
+    from wal_synth import gen_rc1
+    d = gen_rc1(N, K, k, r1, r2, 68, N + K)
+    c = rc.Rc1(N, K, k, d["T"], d["site_pos"], d["site_sign"], d["alpha24"], d["beta24"],
+               d["U1"], d["V1"], d["s1"], d["U2"], d["V2"], d["s2"])
+    can, prep = wal.wal_rc1_sizes(N, K, k, r1, r2)
+    assert can[0] == rc.scales24_plane(c).size
+    for (U, V, s), idx in (((d["U1"], d["V1"], d["s1"]), (1, 2, 3)), ((d["U2"], d["V2"], d["s2"]), (4, 5, 6))):
+        assert [can[i] for i in idx] == [p.size for p in rc.path_planes(U, V, s)]
+    assert list(prep) == [p.size for p in rc.prepared(c)]
+
+
+@pytest.mark.parametrize("args", [(4, 128, 0, 20, 20), (4, 128, 0, -1, 0), (4, 100, 0, 1, 1), (4, 128, 3, 1, 1)])
+def test_rc1_sizes_reject(args):
+    with pytest.raises(wal.WalError) as e:
+        wal.wal_rc1_sizes(*args)
+    assert e.value.status == wal.WAL_ERR_SHAPE
+
+
+def test_last_error_names_the_reason():
+    """A failing call leaves its reason in the thread's error text, which the
+    binding's exception carries."""
+    with pytest.raises(wal.WalError) as e:
+        wal.wal_rc1_sizes(4, 128, 0, 20, 20)
+    assert "r1 + r2" in wal.wal_last_error()
+    assert "r1 + r2" in str(e.value) and "WAL_ERR_SHAPE" in str(e.value)
