@@ -28,7 +28,7 @@ def stream():
 
 def run_gemv(pm, x_dev):
     w = wal()
-    y = torch.empty(pm.N, dtype=torch.float32, device="cuda")
+    y = torch.full((pm.N,), float("nan"), dtype=torch.float32, device="cuda")
     nb = pm.workspace_bytes(1)
     ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
     w.wal_gemv(pm.desc, x_dev.data_ptr(), y.data_ptr(), ws.data_ptr(), nb, stream())
@@ -39,7 +39,7 @@ def run_gemv(pm, x_dev):
 
 def run_gemm(pm, X_dev, M):
     w = wal()
-    Y = torch.empty((M, pm.N), dtype=torch.float32, device="cuda")
+    Y = torch.full((M, pm.N), float("nan"), dtype=torch.float32, device="cuda")
     nb = pm.workspace_bytes(M)
     ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
     w.wal_gemm_small_m(pm.desc, X_dev.data_ptr(), M, pm.K, Y.data_ptr(), pm.N, ws.data_ptr(), nb, stream())
@@ -49,6 +49,9 @@ def run_gemm(pm, X_dev, M):
 
 
 def assert_parity(y, y_ref, x_bits, alpha_bits, what=""):
+    """Every value finite (outputs start as NaN, so an unwritten one shows) and
+    within the oracle tolerance."""
+    assert np.all(np.isfinite(y)), f"{what}: {int(np.size(y) - np.count_nonzero(np.isfinite(y)))} outputs not finite"
     ok, rel, worst = oracle.check_tolerance(y, y_ref, x_bits, alpha_bits)
     assert ok, f"{what}: rel-L2 {rel:.3e} (<= 1e-5), max-abs ratio {worst:.3e} (<= 1)"
     return rel

@@ -7,6 +7,7 @@ import oracle
 from wal_synth import config_plan, gen_components, gen_matrix, gen_x, body_plan, bf16_bits_from_f32, LAYER_8B
 
 from gpu_util import needs_gpu, wal, device_matrix, device_bf16, assert_parity
+import oracle_pool
 
 pytestmark = [pytest.mark.gpu, needs_gpu]
 
@@ -97,67 +98,55 @@ def test_body_stage_dependency():
     bp.close()
 
 
-def test_body8b_full_sampled():
+def test_body8b_full():
     """The full 252-matrix 8B-shaped body pass in the launch configuration the
-    benchmark times; 32 sampled rows of every matrix are checked."""
+    benchmark times.  Every output is checked: the outputs start as NaN, and
+    the oracle computes all rows of every matrix (in a process pool, while the
+    GPU runs)."""
     w = wal()
     specs = config_plan("body8b")
+    xbits = [gen_x(s.K, 1, 2, s.index) for s in specs]
+    refs = oracle_pool.v1_refs_async("body8b", specs, xbits)
     mats, xs, ys = [], [], []
-    rng = np.random.default_rng(12)
-    checks = []
-    for s in specs:
-        c = gen_matrix("body8b", s)
-        x = gen_x(s.K, 1, 2, s.index)
-        rows = np.unique(rng.choice(s.N, 32, replace=False))
-        checks.append((s, rows, oracle.matmul_rows(c, x, rows)[0], x[0], c.alpha))
-        mats.append(device_matrix(c))
+    for s, x in zip(specs, xbits):
+        mats.append(device_matrix(gen_matrix("body8b", s)))
         xs.append(device_bf16(x))
-        ys.append(torch.empty(s.N, dtype=torch.float32, device="cuda"))
-        del c
+        ys.append(torch.full((s.N,), float("nan"), dtype=torch.float32, device="cuda"))
     bp = w.BodyPass(mats, [s.stage for s in specs], xs, ys, M=1)
     bp.run()
     torch.cuda.synchronize()
     _status(bp)
-    for (s, rows, ref, x, alpha), y in zip(checks, ys):
-        assert_parity(y.cpu().numpy().astype(np.float64)[rows], ref, x, alpha, s.name)
+    for s, x, y, (ref, alpha) in zip(specs, xbits, ys, refs.get()):
+        assert_parity(y.cpu().numpy().astype(np.float64).reshape(1, -1), ref, x, alpha, s.name)
     bp.close()
 
 
 @pytest.fixture(scope="module")
 def body27b():
-    """The 448 27B-shaped matrices on the device, with oracle values of 24
-    sampled rows of every matrix for x at M = 1 and M = 4."""
+    """The 448 27B-shaped matrices on the device, with the oracle's outputs
+    for every row of every matrix at M = 1 and M = 4 (computed in a process
+    pool while the matrices are generated and uploaded)."""
     specs = config_plan("body27b")
-    rng = np.random.default_rng(27)
-    mats, checks = [], []
-    for s in specs:
-        c = gen_matrix("body27b", s)
-        rows = np.unique(rng.choice(s.N, 24, replace=False))
-        per_m = {}
-        for M in (1, 4):
-            X = gen_x(s.K, M, 3, 1000 * M + s.index)
-            per_m[M] = (X, oracle.matmul_rows(c, X, rows))
-        checks.append((s, rows, per_m, c.alpha.copy()))
-        mats.append(device_matrix(c))
-        del c
-    return specs, mats, checks
+    X = {M: [gen_x(s.K, M, 3, 1000 * M + s.index) for s in specs] for M in (1, 4)}
+    refs = {M: oracle_pool.v1_refs_async("body27b", specs, X[M]) for M in (1, 4)}
+    mats = [device_matrix(gen_matrix("body27b", s)) for s in specs]
+    return specs, mats, X, refs
 
 
 @pytest.mark.parametrize("M", [1, 4])
-def test_body27b_full_sampled(body27b, M):
+def test_body27b_full(body27b, M):
     """The full 448-matrix 27B-shaped body pass (k by role, 45 matrices with
-    k = 0, 152 with WALB2 r = 8) at batch 1 and 4."""
+    k = 0, 152 with WALB2 r = 8) at batch 1 and 4; every output checked."""
     w = wal()
-    specs, mats, checks = body27b
-    xs = [device_bf16(per_m[M][0]) for (_, _, per_m, _) in checks]
+    specs, mats, X, refs = body27b
+    xs = [device_bf16(x) for x in X[M]]
     ys = [torch.full((M, s.N), float("nan"), dtype=torch.float32, device="cuda") for s in specs]
     bp = w.BodyPass(mats, [s.stage for s in specs], xs, ys, M=M)
     bp.run()
     torch.cuda.synchronize()
     _status(bp)
-    for (s, rows, per_m, alpha), y in zip(checks, ys):
-        X, ref = per_m[M]
-        assert_parity(y.cpu().numpy().astype(np.float64)[:, rows], ref, X, alpha, f"{s.name} M={M}")
+    for s, x, y, (ref, alpha) in zip(specs, X[M], ys, refs[M].get()):
+        assert_parity(y.cpu().numpy().astype(np.float64), ref, x, alpha, f"{s.name} M={M}")
     bp.close()
 
 

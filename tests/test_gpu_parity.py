@@ -13,6 +13,7 @@ import oracle
 from wal_synth import Components, gen_components, gen_x, config_plan, gen_matrix
 
 from golden_io import fixture_names, load
+import oracle_pool
 from gpu_util import (needs_gpu, wal, device_matrix, device_bf16, stream, run_gemv, run_gemm,
                       assert_parity)
 
@@ -140,22 +141,17 @@ def test_small_m_parity_and_columns(M):
             assert np.array_equal(Y[m], run_gemv(pm, device_bf16(X[m])))
 
 
-def _sample_rows(N, rng, count=96):
-    rows = np.unique(np.concatenate([[0, N - 1], rng.choice(N, min(count, N), replace=False)]))
-    return rows
-
-
-def test_layer8b_full_size_sampled():
-    """All seven Qwen3-8B-shaped matrices at full size; every output is
-    computed on the GPU, a sample of rows by the oracle."""
-    rng = np.random.default_rng(7)
-    for spec in config_plan("layer8b"):
-        c = gen_matrix("layer8b", spec)
-        x = gen_x(spec.K, 1, 1, spec.index)[0]
-        y = run_gemv(device_matrix(c), device_bf16(x))
-        rows = _sample_rows(spec.N, rng)
-        ref = oracle.matmul_rows(c, x, rows)[0]
-        assert_parity(y[rows], ref, x, c.alpha, spec.name)
+def test_layer8b_full_size():
+    """All seven Qwen3-8B-shaped matrices at full size; every output of the
+    GPU product is checked against the oracle (all rows, process pool)."""
+    specs = config_plan("layer8b")
+    xs = [gen_x(s.K, 1, 1, s.index) for s in specs]
+    refs = oracle_pool.v1_refs_async("layer8b", specs, xs)
+    ys = []
+    for spec, x in zip(specs, xs):
+        ys.append(run_gemv(device_matrix(gen_matrix("layer8b", spec)), device_bf16(x[0])))
+    for spec, x, y, (ref, alpha) in zip(specs, xs, ys, refs.get()):
+        assert_parity(y.reshape(1, -1), ref, x, alpha, spec.name)
 
 
 def test_validate_detects_corruption():

@@ -14,6 +14,7 @@ import oracle
 from oracle import pq2_oracle as pq
 from wal_synth import config_plan, gen_pq2, gen_x, body_plan, LAYER_8B
 
+import oracle_pool
 from gpu_util import needs_gpu, wal, device_bf16, stream, assert_parity
 
 pytestmark = [pytest.mark.gpu, needs_gpu]
@@ -154,18 +155,16 @@ def test_pq2_body_two_layers_full():
     bp.close()
 
 
-def test_pq2_body8b_full_sampled():
+def test_pq2_body8b_full():
     """The 252-matrix PQ2_0 body pass in the configuration the benchmark times;
-    32 sampled rows of every matrix are checked."""
+    every output checked against the oracle (all rows, process pool)."""
     w = wal()
     specs = config_plan("pq2_body8b")
-    rng = np.random.default_rng(15)
-    mats, xs, ys, checks = [], [], [], []
-    for s in specs:
+    Xs = [gen_x(s.K, 1, 5, s.index) for s in specs]
+    refs = oracle_pool.pq2_refs_async([(s.N, s.K, 5, s.index, X) for s, X in zip(specs, Xs)])
+    mats, xs, ys = [], [], []
+    for s, X in zip(specs, Xs):
         T, d = gen_pq2(s.N, s.K, 5, s.index)
-        X = gen_x(s.K, 1, 5, s.index)
-        rows = np.unique(rng.choice(s.N, 32, replace=False))
-        checks.append((s, rows, pq.matmul_rows(pq.Pq2(s.N, s.K, T, d), X, rows), X, d))
         mats.append(_device(T, d, s.N, s.K))
         xs.append(device_bf16(X))
         ys.append(torch.full((s.N,), float("nan"), dtype=torch.float32, device="cuda"))
@@ -173,6 +172,6 @@ def test_pq2_body8b_full_sampled():
     bp.run()
     torch.cuda.synchronize()
     _status(bp)
-    for (s, rows, ref, X, d), y in zip(checks, ys):
-        assert_parity(y.cpu().numpy().astype(np.float64)[rows].reshape(1, -1), ref, X, d, s.name)
+    for s, X, y, (ref, d) in zip(specs, Xs, ys, refs.get()):
+        assert_parity(y.cpu().numpy().astype(np.float64).reshape(1, -1), ref, X, d, s.name)
     bp.close()

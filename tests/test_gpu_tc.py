@@ -12,6 +12,7 @@ import oracle
 from wal_synth import gen_components, gen_x, config_plan, gen_matrix, bf16_bits_from_f32
 
 from golden_io import fixture_names, load
+import oracle_pool
 from gpu_util import needs_gpu, wal, device_matrix, device_bf16, stream, run_gemm, assert_parity
 
 pytestmark = [pytest.mark.gpu, needs_gpu]
@@ -116,19 +117,13 @@ def test_tc_workspace_is_checked():
     assert e.value.status == w.WAL_ERR_WORKSPACE
 
 
-def _sample_rows(N, rng, count=64):
-    return np.unique(np.concatenate([[0, N - 1], rng.choice(N, min(count, N), replace=False)]))
-
-
 @pytest.mark.parametrize("M", [64, 256, 1024])
-def test_sweep_full_size_sampled(M):
+def test_sweep_full_size(M):
     """gate 4096->12288 and down 12288->4096 (k=8, r=16) at full size: every
-    output on the GPU, a sample of W's rows by the oracle."""
-    rng = np.random.default_rng(M)
-    for spec in config_plan("sweep"):
-        c = gen_matrix("sweep", spec)
-        X = gen_x(spec.K, M, 4, 100 + spec.index)
-        Y = run_gemm(device_matrix(c), device_bf16(X), M)
-        rows = _sample_rows(spec.N, rng)
-        ref = oracle.matmul_rows(c, X, rows)
-        assert_parity(Y[:, rows], ref, X, c.alpha, f"{spec.name} M={M}")
+    output checked against the oracle (all rows, process pool)."""
+    specs = config_plan("sweep")
+    Xs = [gen_x(s.K, M, 4, 100 + s.index) for s in specs]
+    refs = oracle_pool.v1_refs_async("sweep", specs, Xs)
+    Ys = [run_gemm(device_matrix(gen_matrix("sweep", s)), device_bf16(X), M) for s, X in zip(specs, Xs)]
+    for spec, X, Y, (ref, alpha) in zip(specs, Xs, Ys, refs.get()):
+        assert_parity(Y, ref, X, alpha, f"{spec.name} M={M}")
