@@ -139,20 +139,28 @@ int wal_gemv(const wal_matrix* m, const uint16_t* x, float* y, void* ws, size_t 
 int wal_gemm_small_m(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, int ldy,
                      void* ws, size_t ws_bytes, wal_stream_t stream);
 
-/* Y[M][ldy] = X[M][ldx] W^T on the tensor-core path (M >= 17) without a
+/* Y[M][ldy] = X[M][ldx] W^T on the tensor-core path (M >= 8) without a
  * workspace argument.  The model cards have no counterpart to this entry
  * point: it exists for callers that cannot hand the library scratch memory.
  * Its scratch is a fixed array of WAL_NOALLOC_SCRATCH_BYTES in the library's
- * own device memory (one per device, located once per device); a call whose
+ * own device memory (one per device; its address is looked up on every call,
+ * so it always belongs to the current device and context); a call whose
  * scratch need, wal_workspace_bytes(m, M), is larger returns
- * WAL_ERR_WORKSPACE, and M <= 16 returns WAL_ERR_SHAPE.  Nothing is
- * allocated.  Every call on a device uses the same array, so calls that
- * overlap in time on one device (other streams, other host threads) race on
- * it: the caller must order them.  Asynchronous on `stream`; a bounded
- * device wait that gives up is not reported by this entry point. */
+ * WAL_ERR_WORKSPACE, and M < 8 returns WAL_ERR_SHAPE.  Nothing is allocated.
+ * Every call on a device uses the same array, so calls that overlap in time
+ * on one device (other streams, other host threads) race on it: the caller
+ * must order them.  Asynchronous on `stream`.  A bounded device wait that
+ * gives up is recorded in the array's status word: wal_noalloc_status reads
+ * it. */
 #define WAL_NOALLOC_SCRATCH_BYTES (16u << 20)
 int wal_gemm_tc_noalloc(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, int ldy,
                         wal_stream_t stream);
+
+/* Read and clear the status word of the current device's no-alloc scratch
+ * (synchronises `stream`): WAL_OK, or WAL_ERR_TIMEOUT when a bounded device
+ * wait of a wal_gemm_tc_noalloc call since the last read gave up.  Every
+ * wal_gemm_tc_noalloc call clears the word when it starts. */
+int wal_noalloc_status(wal_stream_t stream);
 
 /* Read and clear the device status word in a workspace header (synchronises
  * `stream`).  Every product call clears the word when it starts, so it reports
@@ -181,6 +189,16 @@ int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n_mats,
                   const int32_t* stage_of, const uint16_t* const* xs, float* const* ys, int M,
                   void* ws, size_t ws_bytes, wal_stream_t stream);
 void wal_body_plan_destroy(wal_body_plan* plan);
+
+/* Fault injection for tests of the timeout path (host side only; no GPU fault
+ * is involved).  While the setting is nonzero, body-pass plans built
+ * afterwards (wal_body_pass, wal_pq2_body_pass, wal_rc1_body_pass) get grid
+ * barrier targets that no CTA ever reaches and a 1 ms limit per barrier
+ * wait.  Such a pass ends early: each CTA gives up at its first wait, stops
+ * taking part, waits for its own copies in flight and exits, and
+ * wal_device_status() then returns WAL_ERR_TIMEOUT.  Plans built while the
+ * setting is zero are not affected.  Returns the previous setting. */
+int wal_debug_barrier_fault(int on);
 
 /* ---- PQ2_0: the plain-ternary block format ---------------------------------
  * The WAL2-Ternary-27B card (section on bit widths) describes PQ2_0, the

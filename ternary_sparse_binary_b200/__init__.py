@@ -10,8 +10,8 @@ from ._abi import (  # noqa: F401
     WAL_ERR_UNSUPPORTED, WAL_ERR_TIMEOUT, WAL_MAX_RANK, WAL_MAX_SMALL_M, WAL_NOALLOC_SCRATCH_BYTES,
     WalError, wal_matrix, lib, lib_path, EXPORTED_SYMBOLS,
     wal_packed_sizes, wal_pack_matrix, wal_validate, wal_unpack_matrix, wal_workspace_bytes,
-    wal_gemv, wal_gemm_small_m, wal_gemm_tc_noalloc, wal_device_status, wal_body_workspace_bytes, wal_body_pass,
-    wal_body_plan_destroy, wal_status_string, wal_last_error,
+    wal_gemv, wal_gemm_small_m, wal_gemm_tc_noalloc, wal_noalloc_status, wal_device_status, wal_body_workspace_bytes, wal_body_pass,
+    wal_body_plan_destroy, wal_debug_barrier_fault, wal_status_string, wal_last_error,
     wal_pq2_matrix, wal_pq2_bytes, wal_pq2_pack, wal_pq2_workspace_bytes, wal_pq2_gemm,
     wal_pq2_body_workspace_bytes, wal_pq2_body_pass,
     wal_base3_bytes, wal_base3_pack, wal_base3_convert,

@@ -23,8 +23,8 @@ WAL_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 EXPORTED_SYMBOLS = [
     "wal_packed_sizes", "wal_pack_matrix", "wal_validate", "wal_unpack_matrix",
-    "wal_workspace_bytes", "wal_gemv", "wal_gemm_small_m", "wal_gemm_tc_noalloc", "wal_device_status",
-    "wal_body_workspace_bytes", "wal_body_pass", "wal_body_plan_destroy",
+    "wal_workspace_bytes", "wal_gemv", "wal_gemm_small_m", "wal_gemm_tc_noalloc", "wal_noalloc_status", "wal_device_status",
+    "wal_body_workspace_bytes", "wal_body_pass", "wal_body_plan_destroy", "wal_debug_barrier_fault",
     "wal_pq2_bytes", "wal_pq2_pack", "wal_pq2_workspace_bytes", "wal_pq2_gemm",
     "wal_pq2_body_workspace_bytes", "wal_pq2_body_pass",
     "wal_base3_bytes", "wal_base3_pack", "wal_base3_convert",
@@ -67,7 +67,8 @@ class wal_pq2_matrix(ctypes.Structure):
 
 
 def _load():
-    path = LIB if os.path.exists(LIB) else build()
+    # built in-tree; rebuilt first when a source is newer than the library
+    path = build()
     return ctypes.CDLL(path)
 
 
@@ -87,12 +88,14 @@ lib.wal_gemv.argtypes = [_MP, _vp, _vp, _vp, _sz, _vp]
 lib.wal_gemm_small_m.argtypes = [_MP, _vp, _i, _i, _vp, _i, _vp, _sz, _vp]
 lib.wal_gemm_tc_noalloc.argtypes = [_MP, _vp, _i, _i, _vp, _i, _vp]
 lib.wal_device_status.argtypes = [_vp, _vp]
+lib.wal_noalloc_status.argtypes = [_vp]
 lib.wal_body_workspace_bytes.argtypes = [_MP, _i, _i]
 lib.wal_body_workspace_bytes.restype = _sz
 lib.wal_body_pass.argtypes = [ctypes.POINTER(_vp), _MP, _i, ctypes.POINTER(ctypes.c_int32),
                               ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp, _sz, _vp]
 lib.wal_body_plan_destroy.argtypes = [_vp]
 lib.wal_body_plan_destroy.restype = None
+lib.wal_debug_barrier_fault.argtypes = [_i]
 _PP = ctypes.POINTER(wal_pq2_matrix)
 lib.wal_pq2_bytes.argtypes = [_i, _i]
 lib.wal_pq2_bytes.restype = _sz
@@ -184,6 +187,10 @@ def wal_gemm_tc_noalloc(m, X, M, ldx, Y, ldy, stream):
     return _check(lib.wal_gemm_tc_noalloc(ctypes.byref(m), X, M, ldx, Y, ldy, stream), "wal_gemm_tc_noalloc")
 
 
+def wal_noalloc_status(stream):
+    return _check(lib.wal_noalloc_status(stream), "wal_noalloc_status")
+
+
 def wal_device_status(ws, stream):
     return _check(lib.wal_device_status(ws, stream), "wal_device_status")
 
@@ -206,6 +213,12 @@ def wal_body_pass(plan, mats, stage_of, xs, ys, M, ws, ws_bytes, stream):
 
 def wal_body_plan_destroy(plan):
     lib.wal_body_plan_destroy(plan)
+
+
+def wal_debug_barrier_fault(on):
+    """Fault injection for the timeout tests: body-pass plans built while it is
+    set never pass their first grid barrier.  Returns the previous setting."""
+    return int(lib.wal_debug_barrier_fault(1 if on else 0))
 
 
 def wal_pq2_bytes(N, K):

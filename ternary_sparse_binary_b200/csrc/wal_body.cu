@@ -10,6 +10,8 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include <algorithm>
 #include <vector>
 
@@ -34,6 +36,10 @@ struct wal_body_plan {
 };
 
 namespace {
+
+// Set by wal_debug_barrier_fault: plans built while it is nonzero get a grid
+// barrier that no CTA reaches and a short wait limit.
+std::atomic<int> g_barrier_fault{0};
 
 bool same_matrix(const wal_matrix& a, const wal_matrix& b) {
   return a.N == b.N && a.K == b.K && a.k == b.k && a.r == b.r && a.codes == b.codes && a.sites == b.sites &&
@@ -183,6 +189,11 @@ int body_pass_impl(wal_body_plan** plan, int fmt, const wal_matrix* mats, int n_
     prm.barrier = reinterpret_cast<unsigned int*>(base + kBarrierOffset);
     prm.status = reinterpret_cast<int32_t*>(base);
     prm.fmt = fmt;
+    if (g_barrier_fault.load()) {
+      // fault injection: no CTA reaches a barrier target, and a wait gives up after 1 ms
+      prm.barrier_bias = 1u << 30;
+      prm.wait_ns = 1000000ull;
+    }
 
     e = cudaStreamBeginCapture(p->capture_stream, cudaStreamCaptureModeThreadLocal);
     if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("begin capture: ") + cudaGetErrorString(e));
@@ -233,6 +244,8 @@ extern "C" int wal_body_pass(wal_body_plan** plan, const wal_matrix* mats, int n
   if (!ws || ws_bytes < need) return fail(WAL_ERR_WORKSPACE, "body-pass workspace too small");
   return body_pass_impl(plan, kFmtV1, mats, n_mats, stage_of, xs, ys, M, ws, ws_bytes, (cudaStream_t)stream);
 }
+
+extern "C" int wal_debug_barrier_fault(int on) { return g_barrier_fault.exchange(on ? 1 : 0); }
 
 extern "C" void wal_body_plan_destroy(wal_body_plan* plan) {
   if (!plan) return;

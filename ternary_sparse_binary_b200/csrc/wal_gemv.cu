@@ -165,7 +165,13 @@ int launch_rows(const wal_matrix* m, const uint16_t* X, int ldx, float* Y, int l
 // weight once for all rows (its time hardly grows with M up to a 256-row
 // tile), while the CUDA-core path streams the weights once per row.  On the
 // 8B gate and down shapes at k = 8, r = 16 the two cross between M = 6 and 8.
-constexpr int kTcMinM = 8;
+
+int current_device(int* dev) {
+  const cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (*dev < 0 || *dev >= kMaxDevices) return fail(WAL_ERR_UNSUPPORTED, "device ordinal above 63");
+  return WAL_OK;
+}
 
 size_t product_ws_bytes(const wal_matrix* m, int M) {
   if (M >= kTcMinM) return tc_ws_bytes(m, M);

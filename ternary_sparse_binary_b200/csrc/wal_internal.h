@@ -15,7 +15,11 @@ constexpr int kWordsPerLane = 8;   // one 128-group (8 code words) per lane in t
 constexpr int kSliceCols = 32 * kWordsPerLane * 16;  // 4096 columns per K-slice (one warp)
 constexpr int kLimbWords = 12;     // 3 limbs x 4 slots of uint32 per 16-column code word
 
+constexpr int kMaxDevices = 64;    // device ordinals with their own init state
+
 int fail(int status, const std::string& msg);
+// The current device's ordinal in *dev; WAL_ERR_CUDA or WAL_ERR_UNSUPPORTED (>= kMaxDevices) otherwise.
+int current_device(int* dev);
 int check_shape(int N, int K, int k, int r);
 void sizes_of(int N, int K, int k, int r, size_t out[6]);
 

@@ -79,6 +79,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t
   return false;
 }
 
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+constexpr unsigned long long kDrainWaitNs = 2000000000ull;  // 2 s: limit of one drain wait
+// Wait for a phase that work already issued (a bulk copy of in-bounds memory,
+// or a commit of issued MMAs) completes by itself: used on the way out of a
+// CTA, so that nothing asynchronous is left in flight.  Bounded in time all
+// the same; WAL_ERR_TIMEOUT in *status if it ever ran out.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, int32_t* status) {
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_ns() - t0 > kDrainWaitNs) {
+      if (status) atomicExch(status, (int32_t)WAL_ERR_TIMEOUT);
+      return;
+    }
+}
+
 // ---- bulk copies (no tensor map, no multicast) -------------------------------
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),

@@ -67,7 +67,7 @@ constexpr int kMaxWarps = kMaxThreads / 32;
 constexpr int kMaxXChunks = 8;            // 8-column chunks of x per thread
 constexpr uint32_t kMagic = 0x4B400000u;  // 1.5 * 2^23: adding it rounds |v| < 2^22 to an integer
 constexpr uint32_t kLimbStride = 100;     // words per group in the limb image (96 + 4 pad)
-constexpr uint32_t kBarrierSpin = 1u << 22;  // polls of the grid-barrier counter before giving up
+constexpr unsigned long long kGridWaitNs = 2000000000ull;  // 2 s: far above any grid-barrier wait of a working pass
 // One ring chunk of one warp: rpc rows of codes (32 lanes x 32 B each), then
 // their site bytes (32 x 8 B each + 16 B alignment slack), then their
 // {alpha, beta} words (32 x 4 B each + 16 B slack).  With a single K-slice
@@ -539,6 +539,7 @@ struct RingCtx {
   bool items_global;    // items live in device memory (not kernel parameters)
   int32_t* status;
   unsigned int* barrier;  // grid-barrier counter (body pass)
+  unsigned long long wait_ns;  // limit of one grid-barrier wait
 };
 
 // Consume this warp's rows of the current group (ring positions q, q+1, ...);
@@ -777,15 +778,23 @@ __device__ __forceinline__ void grid_arrive(unsigned int* ctr) {
   __syncthreads();
   if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
 }
-__device__ __forceinline__ void grid_wait(unsigned int* ctr, unsigned int target, int32_t* status) {
-  if (threadIdx.x == 0)
-    for (uint32_t it = 0; ld_acquire(ctr) < target; ++it)
-      if (it >= kBarrierSpin) {
+// The wait is bounded in time (%globaltimer); false on every thread of the CTA
+// when it ran out (WAL_ERR_TIMEOUT recorded).
+__device__ __forceinline__ bool grid_wait(unsigned int* ctr, unsigned int target, int32_t* status,
+                                          unsigned long long limit_ns) {
+  int timed_out = 0;
+  if (threadIdx.x == 0) {
+    const unsigned long long t0 = ptx::global_ns();
+    while (ld_acquire(ctr) < target)
+      if (ptx::global_ns() - t0 > limit_ns) {
         if (status) atomicExch(status, (int32_t)WAL_ERR_TIMEOUT);
+        timed_out = 1;
         break;
       }
-  __syncthreads();
+  }
+  return !__syncthreads_or(timed_out);
 }
+
 
 // wait_target != 0: the grid barrier before this group is still open (this
 // CTA has arrived); the x image and the WALB2 phase-1 products are built
@@ -881,10 +890,12 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
       val = warp_sum(val);
       if (lane == 0) partz[W.s * WAL_MAX_RANK + rho] = val;
     }
-  if (wait_target) grid_wait(R.barrier, wait_target, R.status);
+  // the rows run only after the grid barrier before them (if it is still open) has passed
+  const bool passed = !wait_target || grid_wait(R.barrier, wait_target, R.status, R.wait_ns);
   const uint32_t tab = ptx::smem_u32(area + ap.table) + (uint32_t)g * table_stride(SIGNED_TABLE) * 4u;
-  bool ok = true;
-  if (PQ2) {
+  bool ok = passed;
+  if (!passed) {
+  } else if (PQ2) {
     if (worker) ok = run_rows_pq2(W, R, st, parity, RB, lane, active, lb, xs, gsc, part, lanes);
   } else if (worker) {
     switch (ks) {
@@ -907,6 +918,8 @@ __device__ __forceinline__ bool do_group(const TileRec& t, const RingCtx& R, int
       }
     }
   const bool all_ok = !__syncthreads_or(!ok);
+  // a group whose wait gave up stores nothing (all_ok is the same on every thread)
+  if (!all_ok) return false;
 
   // slices in order, WALB2 phase 2, one store per output
   if (tid < r) {
@@ -970,6 +983,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
   R.items_global = table_mode;
   R.status = prm.status;
   R.barrier = prm.barrier;
+  R.wait_ns = prm.wait_ns ? prm.wait_ns : kGridWaitNs;
   if (lane == 0) {
     for (int st = 0; st < stages; ++st) mbar_init(R.mbar + 8u * st, 1u);
     ptx::mbar_init_fence();
@@ -992,15 +1006,18 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
   bool dead = false;
   for (int j = 0; j < n_groups; ++j) {
     const TileRec t = sched[j];
+    // a CTA whose wait gave up takes no further part: it neither arrives nor
+    // waits (the CTAs that wait for it give up in turn, each after one limit)
+    if (dead) break;
     unsigned int pending = 0;  // target of a grid barrier this CTA has arrived at but not passed
     if (j > 0 && t.stage != sched[j - 1].stage) {
       ++nbar;
       grid_arrive(prm.barrier);
-      pending = nbar * gridDim.x;
+      pending = nbar * gridDim.x + prm.barrier_bias;
       // the x image may be built before the barrier only when the previous
       // stage does not write this group's x (decided on the host)
-      if (t.rows == 0 || dead || !(t.flags & kTileXFree)) {
-        grid_wait(prm.barrier, pending, prm.status);
+      if (t.rows == 0 || !(t.flags & kTileXFree)) {
+        dead = !grid_wait(prm.barrier, pending, prm.status, R.wait_ns);
         pending = 0;
       }
     }
@@ -1011,12 +1028,14 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
                                       : do_group<FMT, false>(t, R, j, st, parity, area, s_z, pending);
     dead = !ok;
   }
-  // never leave with bulk copies in flight: after a wait gave up, wait
-  // (bounded) for the chunks this warp issued but did not consume; they sit
-  // in consecutive slots from the current one
+  // never leave with bulk copies in flight: after a wait gave up, wait for
+  // every chunk this warp issued but did not consume (they sit in consecutive
+  // slots from the current one).  Each is a copy of in-bounds global memory
+  // into this CTA's ring, so its mbarrier phase completes by itself; the wait
+  // is bounded all the same and goes on to the next chunk either way.
   if (lane == 0 && dead)
     for (uint32_t k = R.ps->consumed; k < R.ps->issued; ++k) {
-      if (!mbar_wait(R.mbar + st * 8u, parity, nullptr)) break;
+      ptx::mbar_drain(R.mbar + st * 8u, parity, prm.status);
       if (++st == (uint32_t)stages) {
         st = 0;
         parity ^= 1u;
@@ -1028,33 +1047,43 @@ __global__ void __launch_bounds__(kMaxThreads, 1) stream_kernel(const __grid_con
 // host side
 // ----------------------------------------------------------------------------
 namespace {
-int g_sms = 0;
-int g_max_smem = 0;
-std::once_flag g_once;
-cudaError_t g_err = cudaSuccess;
+// per device: SM count, shared-memory opt-in limit, and the kernels' attribute set once
+struct StreamDev {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+  int sms = 0, max_smem = 0;
+};
+StreamDev g_dev[kMaxDevices];
+
+const StreamDev* dev_state() {
+  int dev = 0;
+  return current_device(&dev) == WAL_OK ? &g_dev[dev] : nullptr;
+}
 }  // namespace
 
 int stream_init() {
-  std::call_once(g_once, [] {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&g_max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(stream_kernel<kFmtV1>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_max_smem - 1024);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(stream_kernel<kFmtPq2>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_max_smem - 1024);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(stream_kernel<kFmtF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_max_smem - 1024);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(stream_kernel<kFmtInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_max_smem - 1024);
-    g_err = e;
+  int dev = 0;
+  int st = current_device(&dev);
+  if (st) return st;
+  StreamDev& d = g_dev[dev];
+  std::call_once(d.once, [&d, dev] {
+    cudaError_t e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    const int lim = d.max_smem - 1024;
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(stream_kernel<kFmtV1>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(stream_kernel<kFmtPq2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(stream_kernel<kFmtF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(stream_kernel<kFmtInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    d.err = e;
   });
-  if (g_err != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("device initialisation: ") + cudaGetErrorString(g_err));
+  if (d.err != cudaSuccess) return fail(WAL_ERR_CUDA, std::string("device initialisation: ") + cudaGetErrorString(d.err));
   return WAL_OK;
 }
 
-int num_sms() { return g_sms > 0 ? g_sms : 148; }
+int num_sms() {
+  const StreamDev* d = dev_state();
+  return d && d->sms > 0 ? d->sms : 148;
+}
 
 int plan_group(StreamItem* items, int n, int K, GroupDesc* out) {
   if (n < 1 || n > kMaxItems) return fail(WAL_ERR_ARG, "a group takes 1..16 products");
@@ -1100,7 +1129,8 @@ int plan_launch(GroupDesc* groups, int n_groups, bool persistent, int fmt, Strea
   for (int j = 0; j < n_groups; ++j) warps = std::max(warps, groups[j].S * groups[j].P);
   if (persistent) warps = kMaxWarps;
   L.threads = 32 * warps;
-  const uint32_t limit = (uint32_t)(g_max_smem > 0 ? g_max_smem : 232448) - 1024u;
+  const StreamDev* dv = dev_state();
+  const uint32_t limit = (uint32_t)(dv && dv->max_smem > 0 ? dv->max_smem : 232448) - 1024u;
   const uint32_t sched_bytes = (uint32_t)align_up((size_t)n_groups * sizeof(TileRec), 128);
   // deepest ring first (rows in flight per warp), fewer copies on a tie
   static const int kRing[6][2] = {{3, 4}, {3, 3}, {2, 4}, {3, 2}, {2, 3}, {2, 2}};

@@ -74,6 +74,8 @@ struct StreamParams {
   uint32_t sched_off;         // shared-memory offset of the CTA's schedule
   uint32_t area_off;          // shared-memory offset of the per-group area
   unsigned int* barrier;      // grid-barrier counter (zeroed before the launch), body pass only
+  unsigned int barrier_bias;  // added to every grid-barrier target (0; the fault-injection hook sets 2^30)
+  unsigned long long wait_ns; // time limit of one grid-barrier wait (0: kGridWaitNs)
   int32_t* status;            // workspace status word (may be NULL)
   int fmt;                    // kFmtV1, kFmtPq2, kFmtF32 or kFmtInt4
 };

@@ -296,9 +296,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
   const uint32_t stage_bytes = kATile * (kHasR ? 2u : 1u) + b_bytes;
   const int S = p.stages;
   const uint32_t bars = base + (uint32_t)S * stage_bytes;
-  // barriers: [S] (unused), a_full[S], empty[S], acc_full.  a_full(s) completes
-  // when the 128 decoders of the stage's team have arrived and the B tile's
-  // bulk copy (one more arrival, with its bytes) has landed.
+  // barriers: b_full[S], a_full[S], empty[S], acc_full.  a_full(s) completes
+  // when the 128 decoders of the stage's team have arrived, b_full(s) when the
+  // B tile's bulk copy has landed (its own barrier, so that the producer can
+  // wait for every copy it issued whatever the decoders do).
+  auto b_full = [&](int s) { return bars + 8u * s; };
   auto a_full = [&](int s) { return bars + 8u * (S + s); };
   auto empty = [&](int s) { return bars + 8u * (2 * S + s); };
   const uint32_t acc_full = bars + 8u * (3 * S);
@@ -321,7 +323,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(a_full(s), 129);  // 128 decoder arrivals + the B tile's arrival with its bytes
+      mbar_init(a_full(s), 128);  // the 128 decoders of the stage's team
+      mbar_init(b_full(s), 1);    // the producer's arrival with the B tile's bytes
       mbar_init(empty(s), 1);
     }
     mbar_init(acc_full, 1);
@@ -341,14 +344,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
     if (lane == 0) {
       // the B tiles are the prep launch's output
       asm volatile("griddepcontrol.wait;" ::: "memory");
+      int issued = 0;
       for (int i = 0; i < n_iter; ++i) {
         const int s = i % S;
         const uint32_t ph = (uint32_t)(i / S) & 1u;
         if (!mbar_wait(empty(s), ph ^ 1u, p.status)) break;
         const char* src = i < KBl ? p.xt + ((size_t)mt * KB + kb0 + i) * b_bytes : p.zt + (size_t)mt * b_bytes;
-        mbar_arrive_expect_tx(a_full(s), b_bytes);
-        bulk_g2s(b_t(s), src, b_bytes, a_full(s));
+        mbar_arrive_expect_tx(b_full(s), b_bytes);
+        bulk_g2s(b_t(s), src, b_bytes, b_full(s));
+        issued = i + 1;
       }
+      // every copy issued lands before the CTA leaves (a slot is refilled only
+      // after its previous copy was consumed, so at most the last S can be
+      // outstanding)
+      for (int i = max(0, issued - S); i < issued; ++i) mbar_drain(b_full(i % S), (uint32_t)(i / S) & 1u, p.status);
     }
   } else if (warp == 1) {
     // ---- MMA issuer ----
@@ -362,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
       int s = 0;
       uint32_t ph = 0u;
       for (int i = 0; i < KBl && ok; ++i) {
-        ok = mbar_wait(a_full(s), ph, p.status);
+        ok = mbar_wait(a_full(s), ph, p.status) && mbar_wait(b_full(s), ph, p.status);
         if (!ok) break;
         tc_fence_after();
         const uint64_t so = (uint64_t)((uint32_t)s * dstage);
@@ -381,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
       if (ok && has_lr) {
         const int s = KBl % S;
         const uint32_t ph = (uint32_t)(KBl / S) & 1u;
-        ok = mbar_wait(a_full(s), ph, p.status);
+        ok = mbar_wait(a_full(s), ph, p.status) && mbar_wait(b_full(s), ph, p.status);
         if (ok) {
           tc_fence_after();
           for (int kk = 0; kk < (2 * p.r + 15) / 16; ++kk)
@@ -390,7 +399,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
           mma_commit(empty(s));
         }
       }
+      // acc_full tracks every MMA issued before it, also after a wait gave up;
+      // tensor memory is released only once they have completed
       mma_commit(acc_full);
+      mbar_drain(acc_full, 0u, p.status);
     }
   } else {
     // ---- decoders, then epilogue ----
@@ -534,25 +546,37 @@ __global__ void __launch_bounds__(256) tc_reduce_kernel(const float* __restrict_
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-std::once_flag g_tc_once;
-cudaError_t g_tc_err = cudaSuccess;
-int g_tc_smem_limit = 0;
+// per device: the shared-memory opt-in limit and the kernels' attribute set once
+struct TcDev {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+  int smem_limit = 0;
+};
+TcDev g_tc_dev[kMaxDevices];
 
 int tc_init() {
-  std::call_once(g_tc_once, [] {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&g_tc_smem_limit, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  int dev = 0;
+  int st = current_device(&dev);
+  if (st) return st;
+  TcDev& d = g_tc_dev[dev];
+  std::call_once(d.once, [&d, dev] {
+    cudaError_t e = cudaDeviceGetAttribute(&d.smem_limit, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    const int lim = d.smem_limit;
     if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_tc_smem_limit);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_tc_smem_limit);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_tc_smem_limit);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, g_tc_smem_limit);
-    g_tc_err = e;
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    d.err = e;
   });
-  if (g_tc_err != cudaSuccess)
-    return fail(WAL_ERR_CUDA, std::string("tensor-core path initialisation: ") + cudaGetErrorString(g_tc_err));
+  if (d.err != cudaSuccess)
+    return fail(WAL_ERR_CUDA, std::string("tensor-core path initialisation: ") + cudaGetErrorString(d.err));
   return WAL_OK;
+}
+
+int tc_smem_limit() {
+  int dev = 0;
+  return current_device(&dev) == WAL_OK && g_tc_dev[dev].smem_limit > 0 ? g_tc_dev[dev].smem_limit : 232448;
 }
 
 uint32_t pow2_ceil(uint32_t v) {
@@ -572,7 +596,7 @@ int plan_tc(const wal_matrix* m, int M, TcPlan* out) {
   const uint32_t b_bytes = (uint32_t)P.M_tile * 128u;
   const uint32_t stage_bytes = kATile * (m->k > 0 ? 2u : 1u) + b_bytes;
   const uint32_t extra = 1024u /*alignment*/ + 8u * (3 * kMaxStages + 1) + 16u + 8u * kMaxTileM;
-  const uint32_t limit = g_tc_smem_limit > 0 ? (uint32_t)g_tc_smem_limit : 232448u;
+  const uint32_t limit = (uint32_t)tc_smem_limit();
   P.stages = (int)std::min<uint32_t>(kMaxStages, (limit - extra) / stage_bytes);
   if (P.stages < 2) return fail(WAL_ERR_UNSUPPORTED, "tensor-core tile does not fit in shared memory");
   P.smem = extra + (uint32_t)P.stages * stage_bytes;

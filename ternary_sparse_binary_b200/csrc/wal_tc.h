@@ -10,6 +10,9 @@
 
 namespace wal {
 
+// Products of this many activation rows or more take the tensor-core path.
+constexpr int kTcMinM = 8;
+
 // Geometry of one tensor-core call.
 struct TcPlan {
   int n_tiles_n;  // 128-row tiles of W

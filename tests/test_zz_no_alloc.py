@@ -54,5 +54,26 @@ def test_limits_are_enforced():
         w.wal_gemm_tc_noalloc(pm.desc, X.data_ptr(), 1024, 12288, Y.data_ptr(), 128, stream())
     assert e.value.status == w.WAL_ERR_WORKSPACE
     with pytest.raises(w.WalError) as e:
-        w.wal_gemm_tc_noalloc(pm.desc, X.data_ptr(), 16, 12288, Y.data_ptr(), 128, stream())
+        w.wal_gemm_tc_noalloc(pm.desc, X.data_ptr(), 7, 12288, Y.data_ptr(), 128, stream())
     assert e.value.status == w.WAL_ERR_SHAPE
+
+
+@pytest.mark.parametrize("M", [8, 16])
+def test_smallest_tensor_batches(M):
+    """M = 8 and 16 take the tensor-core path in wal_gemm_small_m; the no-alloc
+    entry accepts them and gives the same bits."""
+    c = gen_components(300, 1024, 4, 8, config_id=74)
+    pm = device_matrix(c)
+    X = gen_x(1024, M, 74, M)
+    assert np.array_equal(run_noalloc(pm, device_bf16(X), M), run_gemm(pm, device_bf16(X), M))
+
+
+def test_status_reader():
+    """wal_noalloc_status reads (and clears) the scratch status word: OK after
+    calls that completed."""
+    w = wal()
+    pm = device_matrix(gen_components(256, 512, 8, 4, config_id=75))
+    X = gen_x(512, 32, 75, 0)
+    run_noalloc(pm, device_bf16(X), 32)
+    w.wal_noalloc_status(stream())  # raises WalError on anything but WAL_OK
+    w.wal_noalloc_status(stream())
