@@ -1,19 +1,25 @@
 #!/usr/bin/env python3
-"""Benchmark: one 8B-shaped body pass (252 direct-packed matrices, batch 1) per step.
+"""Benchmark of the direct-packed body-matrix product on one B200 (or N replicas).
 
-Default run (one GPU):  python bench.py
-Replicas on N GPUs:     python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N
-Oracle (CPU) arm:       python bench.py --impl reference
-Second workload:        python bench.py --workload pq2_body8b   (the same 252 shapes as
-                        plain-ternary PQ2_0 blocks, 34 bytes per 128 weights)
+    python bench.py                         # the 8B-shaped body pass at batch 1 (default)
+    python bench.py --workload layer8b      # one 8B decoder layer (7 products, 4 stages)
+    python bench.py --workload body27b --batch 4
+    python bench.py --workload pq2_body8b   # the 252 shapes of body8b as PQ2_0 blocks
+    python bench.py --workload sweep --matrix down --batch 64
+    python bench.py --workload format --case int4_head
+    python bench.py --impl reference        # the FP64 oracle on the host cores
+    python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N   # N replicas
 
-Prints ONE JSON line (rank 0).  The metric is microseconds per body pass at
-batch 1 (lower is better) together with the weight stream in GB/s against the
-measured HBM copy bandwidth.
+One step is one pass of the workload: a body pass (one CUDA graph holding a
+header clear and one persistent cooperative launch), or one product call, or
+one format-kernel call.  W untimed warm-up steps, then K steps timed with CUDA
+events on the launching stream; rank 0 prints ONE JSON line.  Workloads whose
+inputs fit in L2 (layer8b, sweep, format) flush L2 (a 256 MiB write, outside
+the timed events) before every step; the body passes stream 2.4-8 GB of
+weights per step, far more than the 126 MB L2.
 """
 import argparse
 import json
-import math
 import os
 import subprocess
 import sys
@@ -25,14 +31,16 @@ sys.path.insert(0, ROOT)
 
 import numpy as np  # noqa: E402
 
-METRIC = "µs per 8B body pass (batch 1) + weight GB/s as % of B200 HBM roofline"
-UNIT = "us/pass"
-WORKLOAD = "body8b"
+HEADLINE_METRIC = "µs per 8B body pass (batch 1) + weight GB/s as % of B200 HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, DGX figure
+BODY_WORKLOADS = ("body8b", "layer8b", "body27b", "pq2_body8b")
+FORMAT_CASES = ("base3", "pq2_gate", "pq2_down", "pq2_27b_up", "int4_head", "rc1_gate")
+DEFAULT_STEPS = {"body8b": 200, "layer8b": 200, "body27b": 50, "pq2_body8b": 200, "sweep": 50, "format": 20}
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None,
@@ -40,35 +48,77 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["wal", "reference"], default="wal")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-matrices", type=int, default=4)
-    ap.add_argument("--workload", choices=["body8b", "pq2_body8b"], default="body8b")
-    a = ap.parse_args()
+    ap.add_argument("--workload", choices=list(BODY_WORKLOADS) + ["sweep", "format"], default="body8b")
+    ap.add_argument("--batch", type=int, default=None, help="activation rows M (default 1; the sweep takes 1..1024)")
+    ap.add_argument("--matrix", choices=["gate", "down"], default="gate", help="sweep: which matrix")
+    ap.add_argument("--case", choices=list(FORMAT_CASES), default="int4_head", help="format: which kernel")
+    a = ap.parse_args(argv)
     if a.steps is None:
-        a.steps = 20 if a.impl == "reference" else 200
-    global WORKLOAD
-    WORKLOAD = a.workload
+        a.steps = 20 if a.impl == "reference" else DEFAULT_STEPS[a.workload]
+    if a.batch is None:
+        a.batch = 1
+    if a.workload == "format":
+        a.batch = 1
+    if a.workload in BODY_WORKLOADS and not 1 <= a.batch <= 16:
+        ap.error("a body pass takes 1 <= --batch <= 16")
+    if a.workload == "pq2_body8b" and a.batch != 1:
+        ap.error("pq2_body8b runs at batch 1")
     return a
 
 
-def is_pq2():
-    return WORKLOAD == "pq2_body8b"
+def metric_of(a):
+    """(metric, unit) of the run: the headline metric for the default workload."""
+    M = a.batch
+    if a.workload == "body8b" and M == 1:
+        return HEADLINE_METRIC, "us/pass"
+    if a.workload == "body8b":
+        return f"µs per 8B body pass (batch {M}) + weight GB/s as % of B200 HBM roofline", "us/pass"
+    if a.workload == "layer8b":
+        return f"µs per 8B decoder layer (7 products, batch {M}) + weight GB/s as % of B200 HBM roofline", "us/layer"
+    if a.workload == "body27b":
+        return f"µs per 27B-shaped body pass (batch {M}) + weight GB/s as % of B200 HBM roofline", "us/pass"
+    if a.workload == "pq2_body8b":
+        return "µs per 8B body pass in PQ2_0 blocks (batch 1) + weight GB/s as % of B200 HBM roofline", "us/pass"
+    if a.workload == "sweep":
+        what = "HBM GB/s" if M < 64 else "tensor TFLOP/s"
+        return f"µs per 8B {a.matrix} product (k=8, r=16) at batch {M} + {what} against the B200 roofline", "us/product"
+    return f"µs per call of the {a.case} format kernel + GB/s against the B200 HBM roofline", "us/call"
 
 
-def workload_text():
-    if is_pq2():
+def workload_text(a):
+    M = a.batch
+    stages = "one CUDA graph holding one persistent cooperative launch, dependency stages separated by grid barriers"
+    if a.workload == "body8b":
+        return (f"8B-shaped body pass: 36 layers x 7 matrices (q,k,v,o 4096-wide; gate/up 4096->12288; "
+                f"down 12288->4096), k=8 sites per 128-group, 213 of 252 with WALB2 r=8, batch {M}, 144 stages, "
+                + stages)
+    if a.workload == "layer8b":
+        return (f"one 8B-shaped decoder layer: q,k,v,o (4096-wide), gate/up 4096->12288, down 12288->4096, k=8, "
+                f"WALB2 r=8 on all seven, batch {M}, 4 stages ([q,k,v] [o] [gate,up] [down]), " + stages)
+    if a.workload == "body27b":
+        return (f"27B-shaped body: 64 layers x 7 matrices (q,k,v,o 5120->5120; gate/up 5120->17408; down "
+                f"17408->5120), k by role (MLP 8, q/k/v 4, o 2, a seeded 45 forced to 0), a seeded 152 of 448 with "
+                f"WALB2 r=8, batch {M}, 256 stages, " + stages)
+    if a.workload == "pq2_body8b":
         return ("8B-shaped body pass in PQ2_0: 36 layers x 7 plain-ternary matrices (q,k,v,o 4096-wide; gate/up "
                 "4096->12288; down 12288->4096), 34-byte blocks (FP16 scale + 32 code bytes) per 128 weights, "
-                "batch 1, one CUDA graph holding one persistent cooperative launch, 144 dependency stages "
-                "separated by grid barriers")
-    return ("8B-shaped body pass: 36 layers x 7 matrices (q,k,v,o 4096-wide; gate/up 4096->12288; "
-            "down 12288->4096), k=8 sites per 128-group, 213 of 252 with WALB2 r=8, batch 1, "
-            "one CUDA graph holding one persistent cooperative launch, 144 dependency stages "
-            "separated by grid barriers")
+                "batch 1, 144 stages, " + stages)
+    if a.workload == "sweep":
+        shape = "gate 4096->12288" if a.matrix == "gate" else "down 12288->4096"
+        path = "CUDA-core decode-GEMV" if M < 8 else "tensor-core path (decode to FP16 tiles + tcgen05.mma)"
+        return f"one product of the 8B {shape} matrix, k=8, WALB2 r=16, batch {M}, {path}"
+    return {"base3": "base-3 -> layout-v1 conversion of a 32768 x 16384 matrix (wal_base3_convert)",
+            "pq2_gate": "PQ2_0 product, 8B gate 4096->12288, batch 1 (wal_pq2_gemm)",
+            "pq2_down": "PQ2_0 product, 8B down 12288->4096, batch 1 (wal_pq2_gemm)",
+            "pq2_27b_up": "PQ2_0 product, 27B up 5120->17408, batch 1 (wal_pq2_gemm)",
+            "int4_head": "INT4/g128 LM head of an 8B model, 4096->151936, batch 1 (wal_int4_gemm)",
+            "rc1_gate": "prepared RC1 product, 8B gate 4096->12288, k=8, two WALB2 paths of rank 4, batch 1 "
+                        "(wal_rc1_gemm)"}[a.case]
 
 
-def seed_id():
+def seed_of(workload):
     from wal_synth import workload_id
-    return workload_id(WORKLOAD)
+    return workload_id(workload)
 
 
 def dist_env():
@@ -76,13 +126,26 @@ def dist_env():
 
 
 def measured_peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    """(copy GB/s, bf16 burst TFLOP/s, bf16 sustained TFLOP/s, 'measured' | 'fallback')."""
     try:
-        with open(p) as fh:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
             d = json.load(fh)
-        return float(d["hbm_gbs"]), "measured"
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), \
+            "measured"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def blas_text():
+    try:
+        from threadpoolctl import threadpool_info
+        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            i = info[0]
+            return f"{i.get('internal_api')} {i.get('version')}", int(i.get("num_threads", 1))
+    except Exception:
+        pass
+    return "unknown", os.cpu_count() or 1
 
 
 # ---------------------------------------------------------------------------
@@ -196,74 +259,459 @@ class ClockSampler:
                 "window_ms": round(1e3 * (rows[-1][0] - rows[0][0]), 1)}
 
 
+
 # ---------------------------------------------------------------------------
-# workload
+# algorithmic sizes
 # ---------------------------------------------------------------------------
-def weight_bytes(s):
-    """Algorithmic (payload) bytes of one matrix, before the 16-byte padding.
-    Layout v1: codes N K / 4, sites N G k, scales N G (4 | 2), U N ceil(r/32) 4,
-    V r K / 8, per-rank scales 2 r.  PQ2_0: 34 bytes per 128 weights."""
-    G = s.K // 128
-    if is_pq2():
-        return s.N * G * 34
-    return (s.N * s.K // 4 + s.N * G * s.k + s.N * G * (4 if s.k else 2) + s.N * ((s.r + 31) // 32) * 4
-            + s.r * s.K // 8 + 2 * s.r)
+def weight_bytes(N, K, k, r):
+    """Payload bytes of one layout-v1 matrix, before the 16-byte padding:
+    codes N K / 4, sites N G k, scales N G (4 | 2), U N ceil(r/32) 4, V r K / 8,
+    per-rank scales 2 r."""
+    G = K // 128
+    return N * K // 4 + N * G * k + N * G * (4 if k else 2) + N * ((r + 31) // 32) * 4 + r * K // 8 + 2 * r
 
 
-def algorithmic_bytes(specs):
-    wbytes = sum(weight_bytes(s) for s in specs)
-    io = sum(2 * s.K + 4 * s.N for s in specs)
-    return wbytes, io
+def pq2_bytes(N, K):
+    """PQ2_0: 34 bytes per 128 weights (FP16 scale + 32 code bytes)."""
+    return N * (K // 128) * 34
 
 
-def build_workload(device):
-    import torch
-    import ternary_sparse_binary_b200 as wal
+def product_flops(N, K, k, r, M):
+    """Algorithmic FLOPs of one product: the ternary dot, the sites and WALB2."""
+    G = K // 128
+    return 2 * M * N * K + 2 * M * N * G * k + 2 * M * r * (N + K)
+
+
+def issued_tensor_flops(N, K, k, M):
+    """What the tensor-core path executes (M >= 8): two K passes over the FP16
+    planes (ternary and residual; one without sites) and the WALB2 MMA (K = 64)."""
+    return 2 * (2 if k else 1) * M * N * K + 2 * M * N * 64
+
+
+# ---------------------------------------------------------------------------
+# the oracle's sample (CPU only): the reference arm and cpu_baseline
+# ---------------------------------------------------------------------------
+def oracle_units(a):
+    """The oracle's bounded sample of the workload and the weight count of one
+    whole step: ([(name, weights, prepare)], step weights).  prepare() builds
+    the packed bytes and x outside the timed region and returns go(), which
+    runs the oracle as it stands: its own unpacker on the packed bytes, dense
+    FP64 W, one matmul.  Body workloads sample layer 0's seven matrices (every
+    layer of a workload has the same shapes); the sweep samples its one product."""
+    import oracle
+    from oracle import pq2_oracle
     from wal_synth import config_plan, gen_matrix, gen_pq2, gen_x
-    specs = config_plan(WORKLOAD)
-    mats = []
-    t0 = time.time()
-    for s in specs:
-        if is_pq2():
-            T, d = gen_pq2(s.N, s.K, seed_id(), s.index)
-            mats.append(wal.Pq2Matrix(wal.pack_pq2_host(T, d, s.N, s.K), s.N, s.K, device=device))
-            del T, d
+    M = a.batch
+    if a.workload == "format":
+        return [], 0
+    plan = "sweep" if a.workload == "sweep" else a.workload
+    specs = config_plan(plan)
+    if a.workload == "sweep":
+        specs = [s for s in specs if s.name == a.matrix]
+        sample = specs
+    else:
+        sample = [s for s in specs if s.layer == 0]
+    cid = seed_of(plan)
+    units = []
+    for s in sample:
+        if a.workload == "pq2_body8b":
+            def prepare(s=s):
+                T, d = gen_pq2(s.N, s.K, cid, s.index)
+                buf = pq2_oracle.pack(pq2_oracle.Pq2(s.N, s.K, T, d))
+                X = gen_x(s.K, M, cid, s.index)
+                return lambda: pq2_oracle.matmul(pq2_oracle.unpack(buf, s.N, s.K), X)
         else:
-            c = gen_matrix(WORKLOAD, s)
-            mats.append(wal.PackedMatrix(wal.pack_host(c), s.N, s.K, s.k, s.r, device=device))
-            del c
-    setup_s = time.time() - t0
-    xoff, yoff = [0], [0]
-    for s in specs:
-        xoff.append(xoff[-1] + s.K)
-        yoff.append(yoff[-1] + s.N)
-    x_host = np.concatenate([gen_x(s.K, 1, seed_id(), s.index)[0] for s in specs]).view(np.int16)
-    x_pinned = torch.from_numpy(x_host).pin_memory()
-    x_dev = x_pinned.to(device)
-    y_dev = torch.empty(yoff[-1], dtype=torch.float32, device=device)
-    y_pinned = torch.empty(yoff[-1], dtype=torch.float32).pin_memory()
-    xs = [x_dev[xoff[i]:xoff[i + 1]] for i in range(len(specs))]
-    ys = [y_dev[yoff[i]:yoff[i + 1]] for i in range(len(specs))]
-    bp = wal.BodyPass(mats, [s.stage for s in specs], xs, ys, M=1, device=device)
-    return dict(specs=specs, mats=mats, bp=bp, x_dev=x_dev, y_dev=y_dev, x_pinned=x_pinned,
-                y_pinned=y_pinned, setup_s=setup_s)
+            def prepare(s=s):
+                bufs = oracle.pack(gen_matrix(plan, s))
+                X = gen_x(s.K, M, cid, s.index)
+                return lambda: oracle.matmul(oracle.unpack(bufs, s.N, s.K, s.k, s.r), X)
+        units.append((s.name, s.N * s.K, prepare))
+    return units, sum(s.N * s.K for s in specs)
 
 
-def count_launches(specs, M=1):
-    """Kernel launches of one body pass: the graph holds a header clear and one
-    persistent launch of the decode-GEMV kernel that runs every stage."""
-    return 1
+def time_unit(prepare):
+    go = prepare()
+    t0 = time.perf_counter()
+    go()
+    return time.perf_counter() - t0
 
 
-def time_gate_product(w, device, reps=20):
-    """Per-launch timing of one product (wal_gemv = one decode-GEMV launch) on
-    the first gate matrix, L2 flushed between launches."""
+def cpu_baseline(a, unit):
+    """The oracle timed once over its whole sample, scaled to one step of the
+    workload by weight count."""
+    units, step_weights = oracle_units(a)
+    if not units:
+        return None
+    ts = [time_unit(p) for _, _, p in units]
+    w_sample = sum(w for _, w, _ in units)
+    blas, cores = blas_text()
+    scale = step_weights / w_sample
+    return {"value": sum(ts) * scale * 1e6, "unit": unit, "cores": cores, "blas": blas, "kind": "oracle",
+            "sample": f"{len(units)} matrices ({', '.join(n for n, _, _ in units)}) at batch {a.batch}: oracle "
+                      f"unpack of the packed bytes + dense FP64 W + matmul, {sum(ts):.1f} s measured"
+                      + (f", scaled x{scale:.0f} by weight count to one step" if abs(scale - 1) > 1e-9 else "")}
+
+
+# ---------------------------------------------------------------------------
+# job timing over replicas
+# ---------------------------------------------------------------------------
+def max_over_ranks(ms, world, device=None):
+    """The largest of the ranks' times (every rank takes part; world 1: itself)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(max_ms, steps, world):
+    """Microseconds per step for the whole job: every rank ran `steps`
+    independent steps (replicas), all inside the slowest rank's time."""
+    return max_ms * 1e3 / (steps * world)
+
+
+# ---------------------------------------------------------------------------
+# the reference arm: the oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(a):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    metric, unit = metric_of(a)
+    units, step_weights = oracle_units(a)
+    if not units:
+        print(json.dumps({"impl": "reference", "unavailable": "format cases have no timed oracle arm"}), flush=True)
+        return 0
+    # step i runs the oracle on sample matrix i mod n (warm-up steps included)
+    per_unit = {}
+    step_s = []
+    t_run0 = time.perf_counter()
+    for i in range(a.warmup + a.steps):
+        name, w, prep = units[i % len(units)]
+        t = time_unit(prep)
+        if i >= a.warmup:
+            per_unit.setdefault(name, (w, []))[1].append(t)
+            step_s.append(t)
+    wall = time.perf_counter() - t_run0
+    covered_w = sum(w for w, _ in per_unit.values())
+    est = sum(np.mean(ts) for _, ts in per_unit.values()) * step_weights / covered_w  # seconds per workload step
+    blas, cores = blas_text()
+    v = est * 1e6
+    cb = {"value": v, "unit": unit, "cores": cores, "blas": blas, "kind": "oracle",
+          "sample": f"step i = oracle on matrix i mod {len(units)} of the sample "
+                    f"({', '.join(n for n, _, _ in units)}), batch {a.batch}: unpack + dense FP64 W + matmul; "
+                    f"value = mean time per sampled matrix summed and scaled x{step_weights / covered_w:.1f} by "
+                    f"weight count to one step of the workload"}
+    line = {"impl": "reference", "metric": metric, "value": v, "unit": unit, "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": float(np.mean(step_s)) * 1e3,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": workload_text(a), "batch": a.batch,
+                                            "wall_s": round(wall, 1)},
+            "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm: workloads
+# ---------------------------------------------------------------------------
+def count_kernels(fn):
+    """This library's kernel launches in one call of fn (a torch.profiler trace
+    of one untimed step; names in namespace wal).  None if no trace could be taken."""
+    import torch
+    try:
+        from torch.profiler import profile, ProfilerActivity
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            fn()
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+        return sum(1 for n in names if "wal::" in n), sorted({n.split("(")[0] for n in names if "wal::" in n})
+    except Exception:
+        return None, []
+
+
+class BodyRun:
+    """A body pass (BodyPass: one CUDA graph) over a workload's matrices, inputs resident in HBM."""
+
+    def __init__(self, a, device):
+        import torch
+        import ternary_sparse_binary_b200 as wal
+        from wal_synth import config_plan, gen_matrix, gen_pq2, gen_x
+        self.a, M = a, a.batch
+        plan = a.workload
+        self.specs = specs = config_plan(plan)
+        cid = seed_of(plan)
+        pq2 = a.workload == "pq2_body8b"
+        t0 = time.time()
+        mats = []
+        for s in specs:
+            if pq2:
+                T, d = gen_pq2(s.N, s.K, cid, s.index)
+                mats.append(wal.Pq2Matrix(wal.pack_pq2_host(T, d, s.N, s.K), s.N, s.K, device=device))
+            else:
+                mats.append(wal.PackedMatrix(wal.pack_host(gen_matrix(plan, s)), s.N, s.K, s.k, s.r, device=device))
+        self.setup_s = time.time() - t0
+        xo, yo = [0], [0]
+        for s in specs:
+            xo.append(xo[-1] + M * s.K)
+            yo.append(yo[-1] + M * s.N)
+        x_host = np.concatenate([gen_x(s.K, M, cid, s.index).reshape(-1) for s in specs]).view(np.int16)
+        self.x_pinned = torch.from_numpy(x_host).pin_memory()
+        self.x_dev = self.x_pinned.to(device)
+        self.y_dev = torch.empty(yo[-1], dtype=torch.float32, device=device)
+        self.y_pinned = torch.empty(yo[-1], dtype=torch.float32).pin_memory()
+        xs = [self.x_dev[xo[i]:xo[i + 1]] for i in range(len(specs))]
+        ys = [self.y_dev[yo[i]:yo[i + 1]] for i in range(len(specs))]
+        self.mats = mats
+        self.bp = wal.BodyPass(mats, [s.stage for s in specs], xs, ys, M=M, device=device)
+        self.flush = torch.empty(256 << 20, dtype=torch.uint8, device=device) if a.workload == "layer8b" else None
+        wb = sum(pq2_bytes(s.N, s.K) if pq2 else weight_bytes(s.N, s.K, s.k, s.r) for s in specs)
+        self.weights = wb
+        self.io = sum(2 * M * s.K + 4 * M * s.N for s in specs)
+        self.h2d, self.d2h = self.x_pinned.numel() * 2, self.y_pinned.numel() * 4
+        self.kernel = "stream_kernel (persistent cooperative launch, one per pass)"
+
+    def step(self):
+        self.bp.run()
+
+    def pre_step(self):
+        if self.flush is not None:
+            self.flush.zero_()
+
+    def e2e_step(self):
+        self.x_dev.copy_(self.x_pinned, non_blocking=True)
+        self.bp.run()
+        self.y_pinned.copy_(self.y_dev, non_blocking=True)
+
+    def check(self):
+        import torch
+        import ternary_sparse_binary_b200 as wal
+        wal.wal_device_status(self.bp.ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+
+    def roofline_bytes(self):
+        return self.weights + self.io
+
+    def config(self):
+        return {"weights_bytes": self.weights, "io_bytes": self.io, "matrices": len(self.specs),
+                "stages": len({s.stage for s in self.specs}), "setup_s": round(self.setup_s, 1)}
+
+    def close(self):
+        self.bp.close()
+
+
+class ProductRun:
+    """One product of the sweep's gate or down matrix (wal_gemv at M = 1, else wal_gemm_small_m)."""
+
+    def __init__(self, a, device):
+        import torch
+        import ternary_sparse_binary_b200 as wal
+        from wal_synth import config_plan, gen_matrix, gen_x
+        self.a, M = a, a.batch
+        self.wal = wal
+        s = next(sp for sp in config_plan("sweep") if sp.name == a.matrix)
+        self.s = s
+        t0 = time.time()
+        self.pm = wal.PackedMatrix(wal.pack_host(gen_matrix("sweep", s)), s.N, s.K, s.k, s.r, device=device)
+        self.setup_s = time.time() - t0
+        x = gen_x(s.K, M, seed_of("sweep"), 100 + s.index).view(np.int16)
+        self.x_pinned = torch.from_numpy(x).pin_memory()
+        self.X = self.x_pinned.to(device)
+        self.Y = torch.empty((M, s.N), dtype=torch.float32, device=device)
+        self.y_pinned = torch.empty((M, s.N), dtype=torch.float32).pin_memory()
+        self.nb = self.pm.workspace_bytes(M)
+        self.ws = torch.empty(self.nb, dtype=torch.uint8, device=device)
+        self.flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+        self.stream = torch.cuda.current_stream()
+        self.weights = weight_bytes(s.N, s.K, s.k, s.r)
+        self.io = 2 * M * s.K + 4 * M * s.N
+        self.h2d, self.d2h = self.x_pinned.numel() * 2, self.y_pinned.numel() * 4
+        self.flops = product_flops(s.N, s.K, s.k, s.r, M)
+        self.issued = issued_tensor_flops(s.N, s.K, s.k, M) if M >= 8 else 0
+        self.kernel = "stream_kernel" if M < 8 else "tc_kernel (with tc_prep_kernel and the split-K sum)"
+
+    def step(self):
+        M, s, w = self.a.batch, self.s, self.wal
+        if M == 1:
+            w.wal_gemv(self.pm.desc, self.X.data_ptr(), self.Y.data_ptr(), self.ws.data_ptr(), self.nb,
+                       self.stream.cuda_stream)
+        else:
+            w.wal_gemm_small_m(self.pm.desc, self.X.data_ptr(), M, s.K, self.Y.data_ptr(), s.N, self.ws.data_ptr(),
+                               self.nb, self.stream.cuda_stream)
+
+    def pre_step(self):
+        self.flush.zero_()
+
+    def e2e_step(self):
+        self.X.copy_(self.x_pinned, non_blocking=True)
+        self.step()
+        self.y_pinned.copy_(self.Y, non_blocking=True)
+
+    def check(self):
+        self.wal.wal_device_status(self.ws.data_ptr(), self.stream.cuda_stream)
+
+    def roofline_bytes(self):
+        return self.weights + self.io
+
+    def config(self):
+        return {"weights_bytes": self.weights, "io_bytes": self.io, "algorithmic_flops": self.flops,
+                "issued_tensor_flops": self.issued or None, "setup_s": round(self.setup_s, 1)}
+
+    def close(self):
+        pass
+
+
+class FormatRun:
+    """One call of a format kernel (the base-3 converter, or a PQ2_0, INT4 or RC1 product)."""
+
+    def __init__(self, a, device):
+        import torch
+        import ternary_sparse_binary_b200 as wal
+        from wal_synth import gen_base3, gen_int4, gen_pq2, gen_rc1, gen_x, Components
+        self.a, self.wal = a, wal
+        self.flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+        st = torch.cuda.current_stream().cuda_stream
+        self.ws = torch.empty(512, dtype=torch.uint8, device=device)
+        self.status_ws = None
+        t0 = time.time()
+        c = a.case
+        if c == "base3":
+            N, K = 32768, 16384
+            T, s = gen_base3(N, K, 6, 1)
+            raw = np.empty(wal.wal_base3_bytes(N, K), np.uint8)
+            wal.wal_base3_pack(T.ctypes.data, N, K, raw.ctypes.data)
+            del T
+            sizes = wal.wal_packed_sizes(N, K, 0, 0)
+            self.inp = torch.from_numpy(raw).pin_memory()
+            b3d, sd = self.inp.to(device), torch.from_numpy(s.view(np.int16).reshape(-1)).to(device)
+            codes = torch.empty(sizes[0], dtype=torch.uint8, device=device)
+            alpha = torch.empty(sizes[2], dtype=torch.uint8, device=device)
+            self.out = codes
+            self.keep = (b3d, sd, alpha)
+            G = K // 128
+            self.bytes = N * ((K + 4) // 5) + 2 * N * G + N * K // 4 + 2 * N * G
+            self.call = lambda: wal.wal_base3_convert(b3d.data_ptr(), sd.data_ptr(), N, K, codes.data_ptr(),
+                                                      alpha.data_ptr(), self.ws.data_ptr(), 512, st)
+            self.dev_in = b3d
+            self.kernel = "base3_convert_kernel"
+        elif c.startswith("pq2"):
+            N, K = {"pq2_gate": (12288, 4096), "pq2_down": (4096, 12288), "pq2_27b_up": (17408, 5120)}[c]
+            T, d = gen_pq2(N, K, 6, N + K)
+            pm = wal.Pq2Matrix(wal.pack_pq2_host(T, d, N, K), N, K, device=device)
+            self.inp = torch.from_numpy(gen_x(K, 1, 6, 1).view(np.int16)).pin_memory()
+            x = self.inp.to(device)
+            y = torch.empty(N, dtype=torch.float32, device=device)
+            nb = pm.workspace_bytes(1)
+            self.ws = torch.empty(nb, dtype=torch.uint8, device=device)
+            self.keep, self.out, self.dev_in = (pm, x), y, x
+            self.bytes = pq2_bytes(N, K) + 2 * K + 4 * N
+            self.call = lambda: wal.wal_pq2_gemm(pm.desc, x.data_ptr(), 1, K, y.data_ptr(), N, self.ws.data_ptr(),
+                                                 nb, st)
+            self.status_ws = self.ws
+            self.kernel = "stream_kernel<PQ2_0>"
+        elif c == "int4_head":
+            N, K = 151936, 4096
+            q, d = gen_int4(N, K, 6, 2)
+            sc, ss = wal.wal_int4_sizes(N, K)
+            cb, sb = np.empty(sc, np.uint8), np.empty(ss, np.uint8)
+            wal.wal_int4_pack(q.ctypes.data, d.ctypes.data, N, K, cb.ctypes.data, sb.ctypes.data)
+            del q
+            cd, sd = torch.from_numpy(cb).to(device), torch.from_numpy(sb).to(device)
+            m = wal.wal_int4_matrix(N, K, cd.data_ptr(), sd.data_ptr())
+            self.inp = torch.from_numpy(gen_x(K, 1, 6, 3).view(np.int16)).pin_memory()
+            x = self.inp.to(device)
+            y = torch.empty(N, dtype=torch.float32, device=device)
+            nb = wal.wal_int4_workspace_bytes(m, 1)
+            self.ws = torch.empty(nb, dtype=torch.uint8, device=device)
+            self.keep, self.out, self.dev_in = (cd, sd, m, x), y, x
+            self.bytes = N * K // 2 + N * (K // 128) * 2 + 2 * K + 4 * N
+            self.call = lambda: wal.wal_int4_gemm(m, x.data_ptr(), 1, K, y.data_ptr(), N, self.ws.data_ptr(), nb, st)
+            self.status_ws = self.ws
+            self.kernel = "stream_kernel<INT4>"
+        else:  # rc1_gate
+            N, K, k, r1, r2 = 12288, 4096, 8, 4, 4
+            dd = gen_rc1(N, K, k, r1, r2, 6, 4)
+            G = K // 128
+            z16 = np.zeros((N, G), np.uint16)
+            base = wal.pack_host(Components(N, K, k, 0, dd["T"], dd["site_pos"], dd["site_sign"], z16, z16,
+                                            np.zeros((N, 0), np.int8), np.zeros((K, 0), np.int8),
+                                            np.zeros(0, np.uint16)))
+
+            def pad(v):
+                return np.concatenate([np.ascontiguousarray(v).reshape(-1).view(np.uint8),
+                                       np.zeros((-v.nbytes) % 16, np.uint8)])
+            paths = []
+            for U, V, s in ((dd["U1"], dd["V1"], dd["s1"]), (dd["U2"], dd["V2"], dd["s2"])):
+                pb = wal.pack_host(Components(N, K, 0, U.shape[1], np.zeros((N, K), np.int8),
+                                              np.zeros((N, G, 0), np.uint8), np.zeros((N, G, 0), np.int8), z16, z16,
+                                              U, V, np.zeros(U.shape[1], np.uint16)))
+                paths.append((U.shape[1], pb[3], pb[4], pad(s)))
+            m = wal.Rc1Matrix.prepare(base[0], base[1], pad(np.concatenate([dd["alpha24"], dd["beta24"]], axis=2)),
+                                      paths[0], paths[1], N, K, k)
+            self.inp = torch.from_numpy(gen_x(K, 1, 6, 5).view(np.int16)).pin_memory()
+            x = self.inp.to(device)
+            y = torch.empty(N, dtype=torch.float32, device=device)
+            nb = m.workspace_bytes(1)
+            self.ws = torch.empty(nb, dtype=torch.uint8, device=device)
+            self.keep, self.out, self.dev_in = (m, x), y, x
+            r = r1 + r2
+            self.bytes = N * K // 4 + N * G * k + N * G * 8 + N * 4 + r * K // 8 + 4 * r + 2 * K + 4 * N
+            self.call = lambda: wal.wal_rc1_gemm(m.desc, x.data_ptr(), 1, K, y.data_ptr(), N, self.ws.data_ptr(),
+                                                 nb, st)
+            self.status_ws = self.ws
+            self.kernel = "stream_kernel<RC1 FP32 scales>"
+        self.setup_s = time.time() - t0
+        self.out_pinned = torch.empty(self.out.numel(), dtype=self.out.dtype).pin_memory()
+        self.h2d, self.d2h = self.inp.numel() * self.inp.element_size(), self.out.numel() * self.out.element_size()
+        self.weights, self.io = self.bytes, 0
+
+    def step(self):
+        self.call()
+
+    def pre_step(self):
+        self.flush.zero_()
+
+    def e2e_step(self):
+        self.dev_in.copy_(self.inp, non_blocking=True)
+        self.call()
+        self.out_pinned.copy_(self.out.reshape(-1), non_blocking=True)
+
+    def check(self):
+        import torch
+        if self.status_ws is not None:
+            self.wal.wal_device_status(self.status_ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+
+    def roofline_bytes(self):
+        return self.bytes
+
+    def config(self):
+        return {"bytes_per_call": self.bytes, "setup_s": round(self.setup_s, 1)}
+
+    def close(self):
+        pass
+
+
+def make_run(a, device):
+    if a.workload in BODY_WORKLOADS:
+        return BodyRun(a, device)
+    if a.workload == "sweep":
+        return ProductRun(a, device)
+    return FormatRun(a, device)
+
+
+def time_gate_launch(run, device, reps=20):
+    """Second roofline entry for the 8B body workloads at batch 1: one product
+    call (wal_gemv or wal_pq2_gemm, one stream_kernel launch) on the pass's
+    first gate matrix, L2 flushed between launches."""
     import torch
     import ternary_sparse_binary_b200 as wal
-    idx = next(i for i, s in enumerate(w["specs"]) if s.name.endswith("gate"))
-    s, pm = w["specs"][idx], w["mats"][idx]
-    pq2 = is_pq2()
-    x = w["x_dev"][: s.K]
+    idx = next(i for i, s in enumerate(run.specs) if s.name.endswith("gate"))
+    s, pm = run.specs[idx], run.mats[idx]
+    pq2 = run.a.workload == "pq2_body8b"
+    x = run.x_dev[sum(sp.K for sp in run.specs[:idx]):][: s.K]
     y = torch.empty(s.N, dtype=torch.float32, device=device)
     nb = pm.workspace_bytes(1)
     ws = torch.empty(nb, dtype=torch.uint8, device=device)
@@ -283,121 +731,30 @@ def time_gate_product(w, device, reps=20):
         e1.synchronize()
         if i >= 3:
             durs.append(e0.elapsed_time(e1) * 1e-3)
-    wbytes = weight_bytes(s) + 2 * s.K + 4 * s.N
+    wal.wal_device_status(ws.data_ptr(), stream.cuda_stream)
+    nbytes = (pq2_bytes(s.N, s.K) if pq2 else weight_bytes(s.N, s.K, s.k, s.r)) + 2 * s.K + 4 * s.N
     dur = float(np.mean(durs))
-    what = f"{s.name} {s.K}->{s.N} PQ2_0" if pq2 else f"{s.name} {s.K}->{s.N} k={s.k} r={s.r}"
-    return {"matrix": what, "bytes_per_launch": wbytes,
-            "us_per_launch": dur * 1e6, "gbs": wbytes / dur / 1e9}
+    return {"kernel": "stream_kernel (single product launch)",
+            "launch": f"{s.name} {s.K}->{s.N}" + (" PQ2_0" if pq2 else f" k={s.k} r={s.r}"),
+            "bytes_per_launch": nbytes, "us_per_launch": dur * 1e6, "achieved": nbytes / dur / 1e9}
 
 
-def load_traffic(kernel="stream_kernel"):
-    """Traffic per launch from the committed ncu summary, if it was taken on
-    the current kernel source (and the workload's format)."""
-    if is_pq2():
-        kernel = "stream_kernel_pq2"
+def load_traffic(a):
+    """DRAM bytes per launch of the roofline kernel from the committed ncu
+    summary, if it was taken on the current kernel source and this workload."""
     import hashlib
-    p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
-        with open(p) as fh:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
             d = json.load(fh)
         src = os.path.join(ROOT, "ternary_sparse_binary_b200", "csrc", "wal_stream.cu")
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        if d.get("source_sha256_16") != h:
+        if d.get("source_sha256_16") != hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]:
             return None
-        return d.get(kernel)
+        return d.get("per_launch", {}).get(f"{a.workload}/M{a.batch}")
     except Exception:
         return None
 
 
-def cpu_baseline(specs, n_sample):
-    """The FP64 oracle as it stands on a bounded sample of the body pass:
-    n_sample matrices (one of each role, cycling), scaled to a full pass by
-    weight count."""
-    import oracle
-    from oracle import pq2_oracle
-    from wal_synth import gen_matrix, gen_pq2, gen_x
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count() or 1
-    roles_seen, sample = set(), []
-    for s in specs:
-        role = s.name.split(".")[1]
-        if role not in roles_seen:
-            roles_seen.add(role)
-            sample.append(s)
-        if len(sample) >= n_sample:
-            break
-    t_total, w_sample = 0.0, 0
-    for s in sample:
-        x = gen_x(s.K, 1, seed_id(), s.index)[0]
-        if is_pq2():
-            T, d = gen_pq2(s.N, s.K, seed_id(), s.index)
-            buf = pq2_oracle.pack(pq2_oracle.Pq2(s.N, s.K, T, d))
-            t0 = time.perf_counter()
-            pq2_oracle.matmul(pq2_oracle.unpack(buf, s.N, s.K), x.reshape(1, -1))
-        else:
-            c = gen_matrix(WORKLOAD, s)
-            t0 = time.perf_counter()
-            oracle.matvec(c, x)
-        t_total += time.perf_counter() - t0
-        w_sample += s.N * s.K
-    w_all = sum(s.N * s.K for s in specs)
-    us_per_pass = t_total * (w_all / w_sample) * 1e6
-    return {"value": us_per_pass, "unit": UNIT, "cores": int(cores), "kind": "oracle",
-            "sample": f"{len(sample)} of 252 matrices ({', '.join(x.name for x in sample)}), "
-                      f"{t_total:.1f} s, scaled to a pass by weight count"}
-
-
-# ---------------------------------------------------------------------------
-# job timing over replicas
-# ---------------------------------------------------------------------------
-def max_over_ranks(ms, world, device=None):
-    """The largest of the ranks' times (every rank takes part; world 1: itself)."""
-    if world <= 1:
-        return float(ms)
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
-def job_rate(max_ms, steps, world):
-    """Microseconds per body pass for the whole job: every rank ran `steps`
-    independent passes (replicas), all inside the slowest rank's time."""
-    return max_ms * 1e3 / (steps * world)
-
-
-# ---------------------------------------------------------------------------
-# arms
-# ---------------------------------------------------------------------------
-def run_reference(args):
-    rank, _, world = dist_env()
-    if rank != 0:
-        return 0
-    from wal_synth import config_plan
-    specs = config_plan(WORKLOAD)
-    n = max(1, args.cpu_sample_matrices // 2)
-    vals = []
-    for i in range(args.warmup + args.steps):
-        cb = cpu_baseline(specs, n)
-        if i >= args.warmup:
-            vals.append(cb["value"])
-    v = float(np.mean(vals))
-    cb["value"] = v
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1e3, "higher_is_better": False,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload_text()},
-            "cpu_baseline": cb,
-            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
-    return 0
-
-
-def run_wal(args):
+def run_wal(a):
     import torch
     import torch.distributed as dist
     rank, local_rank, world = dist_env()
@@ -407,111 +764,127 @@ def run_wal(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local_rank))
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
+    metric, unit = metric_of(a)
 
-    w = build_workload(device)
-    specs, bp = w["specs"], w["bp"]
+    run = make_run(a, device)
     stream = torch.cuda.current_stream()
-    wbytes, iobytes = algorithmic_bytes(specs)
-    launches_per_step = count_launches(specs)
-
-    for _ in range(max(3, args.warmup)):
-        bp.run()
+    for _ in range(max(3, a.warmup)):
+        run.pre_step()
+        run.step()
     torch.cuda.synchronize()
+    run.check()
+    n_launch, kernel_names = count_kernels(run.step)
 
+    # timed region: K steps, CUDA events around each step (flushes outside them)
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.05)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
     h_start = time.monotonic()
-    t_start.record(stream)
-    for i in range(args.steps):
+    for i in range(a.steps):
+        run.pre_step()
         ev[i][0].record(stream)
-        bp.run()
+        run.step()
         ev[i][1].record(stream)
-    t_end.record(stream)
     torch.cuda.synchronize()
     h_end = time.monotonic()
     if world > 1:
         dist.barrier()
     clocks.stop()
-    total_ms = t_start.elapsed_time(t_end)
-    per_step = np.array([a.elapsed_time(b) for a, b in ev]) * 1e3  # us
-    total_ms = max_over_ranks(total_ms, world, device)
-    ms_per_step = total_ms / args.steps
-    us_per_pass_job = job_rate(total_ms, args.steps, world)
-    gbs = (wbytes + iobytes) / (ms_per_step * 1e-3) / 1e9
+    run.check()
+    per_step_us = np.array([x.elapsed_time(y) for x, y in ev]) * 1e3
+    total_ms = max_over_ranks(float(per_step_us.sum()) * 1e-3, world, device)
+    ms_per_step = total_ms / a.steps
+    value = job_rate(total_ms, a.steps, world)
 
-    # end to end: pinned host x -> device, body pass, device y -> host, every step
-    h2d = w["x_pinned"].numel() * 2
-    d2h = w["y_pinned"].numel() * 4
+    # end to end through the public API: pinned host inputs -> device, the step, outputs -> pinned host
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        w["x_dev"].copy_(w["x_pinned"], non_blocking=True)
-        bp.run()
-        w["y_pinned"].copy_(w["y_dev"], non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
-    e2e_us = job_rate(e2e_ms, args.steps, world)
+    e2e_us = []
+    for _ in range(a.steps):
+        run.pre_step()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run.e2e_step()
+        e1.record(stream)
+        e1.synchronize()
+        e2e_us.append(e0.elapsed_time(e1) * 1e3)
+    run.check()
+    e2e_ms = max_over_ranks(float(np.sum(e2e_us)) * 1e-3, world, device)
+    e2e_value = job_rate(e2e_ms, a.steps, world)
 
-    kernel = time_gate_product(w, device) if rank == 0 else None
-    peak, peak_kind = measured_peaks()
+    hbm, tfl_burst, tfl_sus, peak_kind = measured_peaks()
+    nbytes = run.roofline_bytes()
+    step_s = float(np.mean(per_step_us)) * 1e-6
+    if a.workload == "sweep" and a.batch >= 64:
+        achieved = run.flops / step_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tfl_burst, "unit": "TFLOP/s",
+                "frac": achieved / tfl_burst, "traffic": None,
+                "peak_kind": f"{peak_kind} cuBLAS bf16 burst (FP16 operands run at the bf16 rate)",
+                "issued_tflops": run.issued / step_s / 1e12, "frac_issued": run.issued / step_s / 1e12 / tfl_burst}
+    else:
+        achieved = nbytes / step_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": load_traffic(a), "peak_kind": f"{peak_kind} copy bandwidth (hbm_gbs)",
+                "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS}
+    roof.update({"kernel": run.kernel, "bytes_per_launch": nbytes,
+                 "us_per_launch": step_s * 1e6,
+                 "timing": "CUDA events around each step on its stream inside the timed region"
+                           + ("; the step's graph also holds a 256-byte header memset" if a.workload in BODY_WORKLOADS
+                              else "")})
+
+    gate = None
+    if rank == 0 and a.workload in ("body8b", "pq2_body8b", "layer8b") and a.batch == 1:
+        gate = time_gate_launch(run, device)
+        gate.update({"bound": "hbm", "peak": hbm, "unit": "GB/s", "frac": gate["achieved"] / hbm})
 
     cb = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_baseline(specs, args.cpu_sample_matrices)
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cb = cpu_baseline(a, unit)
 
     if rank == 0:
-        traffic = load_traffic()
+        launches = n_launch if n_launch is not None else (1 if a.workload in BODY_WORKLOADS else None)
         line = {
-            "metric": METRIC, "value": us_per_pass_job, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",
-            "vs_baseline": None, "dtype": "int32+f32 (dp4a on a 24-bit fixed-point x image, FP32 scales and accumulation)",
+            "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "int32+f32 (dp4a on a 24-bit fixed-point x image, FP32 scales and accumulation)"
+                     if not (a.workload == "sweep" and a.batch >= 8) else
+                     "f16 tensor-core operands (exact ternary/residual planes), f32 accumulation",
             "data": "synthetic",
-            "config": {"workload": workload_text(),
-                       "weights_bytes": wbytes, "io_bytes": iobytes,
-                       "l2": f"inputs larger than L2 ({wbytes / 1e9:.2f} GB of packed weights per pass vs 126 MB L2)",
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "step_us_p10_p50_p90": [float(np.percentile(per_step, q)) for q in (10, 50, 90)],
-                       "weight_gbs": gbs, "setup_s": round(w["setup_s"], 1)},
-            # dominant kernel: stream_kernel, timed per launch on the largest matrix of the pass
-            "roofline": {"bound": "hbm", "achieved": kernel["gbs"], "peak": peak, "unit": "GB/s",
-                         "frac": kernel["gbs"] / peak, "traffic": traffic,
-                         "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS hbm_gbs)",
-                         "kernel": "stream_kernel", "launch": kernel["matrix"],
-                         "bytes_per_launch": kernel["bytes_per_launch"], "us_per_launch": kernel["us_per_launch"],
-                         "timing": "CUDA events around each launch on its stream, L2 flushed between launches"},
-            "pass_roofline": {"achieved": gbs, "unit": "GB/s", "frac": gbs / peak,
-                              "frac_of_nominal_8tbs": gbs / NOMINAL_HBM_GBS,
-                              "scope": "whole body pass (graph): packed weights + x + y per pass / ms per pass"},
-            "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps,
+            "config": dict({"workload": workload_text(a), "batch": a.batch,
+                            "l2": "L2 flushed (256 MiB write) before every step, outside the timed events"
+                            if a.workload not in ("body8b", "body27b", "pq2_body8b") else
+                            f"inputs larger than L2 ({nbytes / 1e9:.2f} GB per step vs 126 MB L2)",
+                            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                            "step_us_p10_p50_p90": [float(np.percentile(per_step_us, q)) for q in (10, 50, 90)]},
+                           **run.config()),
+            "roofline": roof,
+            "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": run.h2d, "d2h_bytes_per_step": run.d2h},
+            "gpu_launches": launches * a.steps if launches is not None else None,
+            "gpu_kernels": kernel_names,
             "clocks": clocks.summary(h_start, h_end),
         }
+        if gate:
+            line["roofline_gate_launch"] = gate
         if cb:
             line["cpu_baseline"] = cb
         print(json.dumps(line), flush=True)
-    bp.close()
+    run.close()
     if world > 1:
         dist.destroy_process_group()
     return 0
 
 
 def main():
-    args = parse()
-    if args.impl == "reference":
-        return run_reference(args)
-    return run_wal(args)
+    a = parse()
+    if a.impl == "reference":
+        return run_reference(a)
+    return run_wal(a)
 
 
 if __name__ == "__main__":
