@@ -98,6 +98,13 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, int32_
     }
 }
 
+// One lane of a converged warp (the same one on every lane's view).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(e));
+  return e != 0;
+}
+
 // ---- bulk copies (no tensor map, no multicast) -------------------------------
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),

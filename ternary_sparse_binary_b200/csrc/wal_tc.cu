@@ -361,19 +361,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
     }
   } else if (warp == 1) {
     // ---- MMA issuer ----
-    if (lane == 0) {
-      const uint32_t idesc = idesc_f16_f32(kRows, (uint32_t)p.M_tile);
-      // descriptors of stage 0; a stage step or a 16-column step only moves
-      // the 14-bit start-address field (address / 16), which never carries
-      const uint64_t da0 = sdesc_sw128(a_t(0)), dr0 = sdesc_sw128(a_r(0)), db0 = sdesc_sw128(b_t(0));
-      const uint32_t dstage = stage_bytes >> 4;
-      bool ok = true;
-      int s = 0;
-      uint32_t ph = 0u;
-      for (int i = 0; i < KBl && ok; ++i) {
-        ok = mbar_wait(a_full(s), ph, p.status) && mbar_wait(b_full(s), ph, p.status);
-        if (!ok) break;
-        tc_fence_after();
+    // The whole warp runs the loop, so its addresses and counters stay
+    // warp-uniform; one elected lane issues the MMAs and commits.  A wait
+    // ends the loop for every lane together (__all_sync).
+    const uint32_t idesc = idesc_f16_f32(kRows, (uint32_t)p.M_tile);
+    // descriptors of stage 0; a stage step or a 16-column step only moves
+    // the 14-bit start-address field (address / 16), which never carries
+    const uint64_t da0 = sdesc_sw128(a_t(0)), dr0 = sdesc_sw128(a_r(0)), db0 = sdesc_sw128(b_t(0));
+    const uint32_t dstage = stage_bytes >> 4;
+    bool ok = true;
+    int s = 0;
+    uint32_t ph = 0u;
+    for (int i = 0; i < KBl && ok; ++i) {
+      ok = __all_sync(0xffffffffu, mbar_wait(a_full(s), ph, p.status) && mbar_wait(b_full(s), ph, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      if (elect_one()) {
         const uint64_t so = (uint64_t)((uint32_t)s * dstage);
 #pragma unroll
         for (int kk = 0; kk < kBlockK / 16; ++kk) {
@@ -382,28 +385,34 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
           if (kHasR) mma_f16(tmem, dr0 + so + 2u * kk, bd, idesc, 1u);
         }
         mma_commit(empty(s));
-        if (++s == S) {
-          s = 0;
-          ph ^= 1u;
-        }
       }
-      if (ok && has_lr) {
-        const int s = KBl % S;
-        const uint32_t ph = (uint32_t)(KBl / S) & 1u;
-        ok = mbar_wait(a_full(s), ph, p.status) && mbar_wait(b_full(s), ph, p.status);
-        if (ok) {
-          tc_fence_after();
-          for (int kk = 0; kk < (2 * p.r + 15) / 16; ++kk)
-            mma_f16(tmem + p.d2_col, sdesc_sw128(a_t(s) + 32u * kk), sdesc_sw128(b_t(s) + 32u * kk), idesc,
-                    kk != 0);
-          mma_commit(empty(s));
-        }
+      __syncwarp();
+      if (++s == S) {
+        s = 0;
+        ph ^= 1u;
       }
-      // acc_full tracks every MMA issued before it, also after a wait gave up;
-      // tensor memory is released only once they have completed
-      mma_commit(acc_full);
-      mbar_drain(acc_full, 0u, p.status);
     }
+    if (ok && has_lr) {
+      const int s2 = KBl % S;
+      const uint32_t ph2 = (uint32_t)(KBl / S) & 1u;
+      ok = __all_sync(0xffffffffu, mbar_wait(a_full(s2), ph2, p.status) && mbar_wait(b_full(s2), ph2, p.status));
+      if (ok) {
+        tc_fence_after();
+        if (elect_one()) {
+          for (int kk = 0; kk < (2 * p.r + 15) / 16; ++kk)
+            mma_f16(tmem + p.d2_col, sdesc_sw128(a_t(s2) + 32u * kk), sdesc_sw128(b_t(s2) + 32u * kk), idesc,
+                    kk != 0);
+          mma_commit(empty(s2));
+        }
+        __syncwarp();
+      }
+    }
+    // acc_full tracks every MMA issued before it, also after a wait gave up;
+    // tensor memory is released only once they have completed
+    if (elect_one()) mma_commit(acc_full);
+    __syncwarp();
+    if (lane == 0) mbar_drain(acc_full, 0u, p.status);
+    __syncwarp();
   } else {
     // ---- decoders, then epilogue ----
     const int h = (warp - 2) >> 2;      // team
