@@ -29,6 +29,12 @@ __device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
 __device__ __forceinline__ void sts16(uint32_t a, uint32_t v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"((uint16_t)v) : "memory");
 }
+// The 16-bit store, done only where `pred` holds (a predicated instruction, no branch).
+__device__ __forceinline__ void sts16_if(bool pred, uint32_t a, uint32_t v) {
+  asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %2, 0;\n @p st.shared.u16 [%0], %1;\n}\n" ::"r"(a),
+               "h"((uint16_t)v), "r"((uint32_t)pred)
+               : "memory");
+}
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));

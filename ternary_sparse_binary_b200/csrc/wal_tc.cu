@@ -285,7 +285,7 @@ __device__ __forceinline__ GroupLoad<KS> load_group(const TcParams& p, int n, in
 }
 
 template <int KS>
-__global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
+__global__ void __launch_bounds__(kThreads, 2) tc_kernel(const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   constexpr bool kHasR = KS > 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -453,14 +453,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcParams p) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) sts128(ar + (((uint32_t)c ^ r7) << 4), make_uint4(0u, 0u, 0u, 0u));
         const uint32_t beta = cur.scales >> 16;
+        // straight-line code with a predicated store per site: the sites of
+        // a warp's rows fall in either half at random, and a branch per site
+        // diverged on every one
 #pragma unroll
         for (int j = 0; j < KS; ++j) {
           const uint32_t b = ((j < 4 ? cur.sites_lo : cur.sites_hi) >> (8 * (j & 3))) & 0xFFu;
-          if (live && ((b >> 6) & 1u) == (uint32_t)h) {
-            const uint32_t pos = b & 63u, jj = pos & 15u;
-            const uint32_t col = (pos & 48u) | ((jj & 3u) << 2) | (jj >> 2);
-            sts16(ar + ((((col >> 3) ^ r7) & 7u) << 4) + 2u * (col & 7u), beta ^ ((b & 0x80u) << 8));
-          }
+          const uint32_t pos = b & 63u, jj = pos & 15u;
+          const uint32_t col = (pos & 48u) | ((jj & 3u) << 2) | (jj >> 2);
+          sts16_if(live && ((b >> 6) & 1u) == (uint32_t)h, ar + ((((col >> 3) ^ r7) & 7u) << 4) + 2u * (col & 7u),
+                   beta ^ ((b & 0x80u) << 8));
         }
       }
       fence_proxy_async_smem();
@@ -605,12 +607,20 @@ int plan_tc(const wal_matrix* m, int M, TcPlan* out) {
   const uint32_t b_bytes = (uint32_t)P.M_tile * 128u;
   const uint32_t stage_bytes = kATile * (m->k > 0 ? 2u : 1u) + b_bytes;
   const uint32_t extra = 1024u /*alignment*/ + 8u * (3 * kMaxStages + 1) + 16u + 8u * kMaxTileM;
-  const uint32_t limit = (uint32_t)tc_smem_limit();
-  P.stages = (int)std::min<uint32_t>(kMaxStages, (limit - extra) / stage_bytes);
-  if (P.stages < 2) return fail(WAL_ERR_UNSUPPORTED, "tensor-core tile does not fit in shared memory");
-  P.smem = extra + (uint32_t)P.stages * stage_bytes;
   const uint32_t d2 = pow2_ceil((uint32_t)P.M_tile);
   P.tmem_cols = std::max(32u, d2 * (m->r > 0 ? 2u : 1u));
+  // Two CTAs per SM when half the tensor memory and half the shared memory
+  // (of the B200's 228 KB per SM, less 1 KB per CTA) hold a CTA with at least
+  // two stages: the two MMA-issuing loops then overlap.  The registers allow
+  // it (launch bounds).  Otherwise one CTA per SM with all the shared memory.
+  const uint32_t limit = (uint32_t)tc_smem_limit();
+  constexpr uint32_t kPairSmem = 233472u / 2u - 1024u;
+  const bool pair = P.tmem_cols <= 256u && kPairSmem >= extra + 2u * stage_bytes;
+  const uint32_t budget = pair ? std::min(limit, kPairSmem) : limit;
+  P.stages = (int)std::min<uint32_t>(kMaxStages, (budget - extra) / stage_bytes);
+  if (P.stages < 2) return fail(WAL_ERR_UNSUPPORTED, "tensor-core tile does not fit in shared memory");
+  P.smem = extra + (uint32_t)P.stages * stage_bytes;
+  P.per_sm = pair ? 2 : 1;
   // K splits: with few row tiles, split K so the grid fills the SMs.  Cost
   // model in microseconds: waves x (K-blocks per split + about 4 of fixed
   // work) x about 1 us per K-block, plus the split sums' traffic (ks partial
@@ -625,7 +635,7 @@ int plan_tc(const wal_matrix* m, int M, TcPlan* out) {
   for (int ks = 1; ks <= std::min(G, 16); ++ks) {
     const int gps = (G + ks - 1) / ks, eff = (G + gps - 1) / gps;
     if (eff != ks) continue;
-    const int waves = (tiles * ks + kPlanSms - 1) / kPlanSms;
+    const int waves = (tiles * ks + kPlanSms * P.per_sm - 1) / (kPlanSms * P.per_sm);
     const double reduce_us = ks > 1 ? (double)(ks + 1) * M * m->N * 4.0 / 3.0e6 : 0.0;
     const double est = (double)waves * (2.0 * gps + 4.0) + reduce_us;
     if (est < best - 1e-9) {

@@ -23,6 +23,7 @@ struct TcPlan {
   int ks, gps;    // K splits and 128-column groups per split
   uint32_t smem;  // dynamic shared memory per CTA
   uint32_t tmem_cols;
+  int per_sm;     // CTAs resident per SM (1 or 2)
   // workspace offsets from the 256-byte aligned base
   size_t off_scal, off_zt, off_xt, off_part, total;
 };
