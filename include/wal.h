@@ -123,8 +123,8 @@ int wal_unpack_matrix(const wal_matrix* m, int8_t* T, uint8_t* site_pos, int8_t*
                       wal_stream_t stream);
 
 /* Scratch bytes wal_gemv (M = 1) / wal_gemm_small_m (any M) need: the
- * 256-byte header for M <= 7, the tensor path's X image, WALB2 operand and
- * split sums from M = 8 on. */
+ * 256-byte header for M <= 4, the tensor path's X image, WALB2 operand and
+ * split sums from M = 5 on. */
 size_t wal_workspace_bytes(const wal_matrix* m, int M);
 
 /* y[N] = W x for one bf16 activation x[K] (batch 1): the decode-GEMV.
@@ -132,21 +132,21 @@ size_t wal_workspace_bytes(const wal_matrix* m, int M);
 int wal_gemv(const wal_matrix* m, const uint16_t* x, float* y, void* ws, size_t ws_bytes,
              wal_stream_t stream);
 
-/* Y[M][ldy] = X[M][ldx] W^T for 1 <= M.  M <= 7 runs the CUDA-core
- * decode-GEMV, one product per activation row in one launch; M >= 8 runs the
+/* Y[M][ldy] = X[M][ldx] W^T for 1 <= M.  M <= 4 runs the CUDA-core
+ * decode-GEMV, one product per activation row in one launch; M >= 5 runs the
  * tensor-core path (bulk copies + tcgen05), which decodes each weight once for
  * up to 256 rows.  ldx >= K and a multiple of 8; ldy >= N. */
 int wal_gemm_small_m(const wal_matrix* m, const uint16_t* X, int M, int ldx, float* Y, int ldy,
                      void* ws, size_t ws_bytes, wal_stream_t stream);
 
-/* Y[M][ldy] = X[M][ldx] W^T on the tensor-core path (M >= 8) without a
+/* Y[M][ldy] = X[M][ldx] W^T on the tensor-core path (M >= 5) without a
  * workspace argument.  The model cards have no counterpart to this entry
  * point: it exists for callers that cannot hand the library scratch memory.
  * Its scratch is a fixed array of WAL_NOALLOC_SCRATCH_BYTES in the library's
  * own device memory (one per device; its address is looked up on every call,
  * so it always belongs to the current device and context); a call whose
  * scratch need, wal_workspace_bytes(m, M), is larger returns
- * WAL_ERR_WORKSPACE, and M < 8 returns WAL_ERR_SHAPE.  Nothing is allocated.
+ * WAL_ERR_WORKSPACE, and M < 5 returns WAL_ERR_SHAPE.  Nothing is allocated.
  * Every call on a device uses the same array, so calls that overlap in time
  * on one device (other streams, other host threads) race on it: the caller
  * must order them.  Asynchronous on `stream`.  A bounded device wait that

@@ -38,7 +38,7 @@ extern "C" int wal_gemm_tc_noalloc(const wal_matrix* m, const uint16_t* X, int M
                                    wal_stream_t stream) {
   int st = check_product_args(m, X, M, ldx, Y, ldy);
   if (st) return st;
-  if (M < kTcMinM) return fail(WAL_ERR_SHAPE, "wal_gemm_tc_noalloc takes M >= 8 (the tensor-core path)");
+  if (M < kTcMinM) return fail(WAL_ERR_SHAPE, "wal_gemm_tc_noalloc takes M >= 5 (the tensor-core path)");
   const size_t need = tc_ws_bytes(m, M);
   if (need == 0 || need > kScratchBytes)
     return fail(WAL_ERR_WORKSPACE, "scratch need above the fixed 16 MiB array");

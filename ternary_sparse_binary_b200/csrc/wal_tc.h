@@ -11,7 +11,11 @@
 namespace wal {
 
 // Products of this many activation rows or more take the tensor-core path.
-constexpr int kTcMinM = 8;
+// Its time hardly grows with M up to a 16-row tile, while the CUDA-core path
+// streams the weights once per row: measured on the 8B gate (down) shape at
+// k = 8, r = 16, M = 4 takes 35.8 (48.1) us on CUDA cores and 42.0 (46.2) on
+// the tensor path, M = 5 42.0 (56.3) against 42.1 (46.1).
+constexpr int kTcMinM = 5;
 
 // Geometry of one tensor-core call.
 struct TcPlan {
