@@ -19,13 +19,14 @@ pytestmark = [pytest.mark.gpu, needs_gpu]
 
 TC_SHAPES = [  # N, K, k, r, M
     (256, 512, 8, 8, 64),
-    (200, 384, 4, 16, 17),     # ragged second row tile; the smallest batch on this path
+    (200, 384, 4, 16, 17),     # ragged second row tile
     (130, 256, 2, 0, 100),     # batch not a multiple of 16
     (128, 1024, 0, 32, 256),   # plain ternary + maximum rank, one full activation tile
     (384, 768, 8, 3, 300),     # two activation tiles, the second ragged
     (64, 128, 8, 1, 33),       # a single group, fewer rows than a tile
     (1000, 2176, 8, 8, 64),
-    (1000, 2176, 8, 8, 8),     # the smallest batch on this path
+    (1000, 2176, 8, 8, 8),
+    (1000, 2176, 8, 8, 5),     # the smallest batch on this path
     (300, 4096, 4, 16, 12),
     (64, 128, 8, 1, 16),
     (12288, 4096, 8, 16, 16),  # the gate shape of the batch sweep
